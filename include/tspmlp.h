@@ -1,0 +1,188 @@
+/*
+ * tspmlp.h -- C ABI of libtspmlp: the column-then-row sharded transformer MLP
+ * on one NVIDIA B200 (sm_100a).
+ *
+ * The operation.  For token rows X[n][d_model]:
+ *
+ *   plain  (TSP_ACT_GELU):   Y = GeLU(X.A).B                     GeLU(z) = z Phi(z)
+ *   gated  (TSP_ACT_SWIGLU): Y = (SiLU(X.W_gate) (*) (X.W_up)).W_down
+ *
+ * "Tensor Parallelism: Splitting the Math" (section "Why the column-then-row
+ * split -- and what happens in attention") defines the plain block and shows
+ * that splitting A by columns and B by rows lets every shard apply the
+ * nonlinearity to values it fully owns; steps 2-6 of its two-GPU walk-through
+ * ("One transformer MLP, split across two GPUs") define the shards and the sum
+ * of their partial outputs.  "Folding Tensor and Sequence Parallelism for
+ * Memory-Efficient Transformer Training & Inference" (Abstract) gives the
+ * gated form and the folded schedule in which weight shards circulate in a
+ * ring while each sequence shard accumulates its partial outputs locally.
+ *
+ * Here the P shards are logical: shard w owns hidden columns
+ * [w d_ff/P, (w+1) d_ff/P) of A (= W_gate) and W_up and the same rows of
+ * B (= W_down).  All shards run on the calling GPU; each shard's partial output
+ * is added into an fp32 accumulator in place, in shard order (no collective).
+ *
+ * Layout and types.  Every matrix is dense and row-major, as in the pages'
+ * product X.A:
+ *   X[n][d_model], A = W_gate[d_model][d_ff], W_up[d_model][d_ff],
+ *   B = W_down[d_ff][d_model], Y[n][d_model], dY[n][d_model].
+ * (torch.nn.Linear stores the transpose of each weight.)
+ * TSP_DT_BF16: X, weights, dY, Y and dX are bfloat16; every product
+ *   accumulates in fp32; the hidden activation is rounded to bf16 once before
+ *   the down projection; weight gradients are fp32.
+ * TSP_DT_F32: everything fp32 (no TF32), plain or gated.
+ *
+ * Ownership.  The caller owns every buffer.  Pointers are device pointers on
+ * the current device unless a function says otherwise.  The library keeps no
+ * state between calls apart from per-device kernel attributes set once and a
+ * device-side error word.  Calls that take no workspace allocate their scratch
+ * with cudaMallocAsync on `stream` and free it on the same stream.
+ *
+ * Errors.  Arguments are validated before anything is launched; a bad call
+ * returns a status and touches nothing.  Kernels bound every wait on the GPU
+ * (about two seconds); a wait that runs out sets the device error word and the
+ * kernel returns early, so a later tsp_poll_device_error() reports
+ * TSP_ERR_TIMEOUT instead of hanging.  All calls are asynchronous on `stream`.
+ */
+#ifndef TSPMLP_H
+#define TSPMLP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TSP_API __attribute__((visibility("default")))
+#else
+#define TSP_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream (layout-compatible with cudaStream_t); NULL is the legacy
+ * default stream. */
+typedef struct CUstream_st* tsp_stream_t;
+
+typedef enum {
+    TSP_OK = 0,
+    TSP_ERR_INVALID_ARG = 1,       /* NULL pointer, non-positive size, bad enum, aliasing */
+    TSP_ERR_UNSUPPORTED_SHAPE = 2, /* d_ff % P, alignment or size limits (see each call) */
+    TSP_ERR_ARCH = 3,              /* current device is not compute capability 10.0 */
+    TSP_ERR_CUDA = 4,              /* a CUDA runtime call or launch failed */
+    TSP_ERR_TIMEOUT = 5,           /* a bounded device-side wait ran out */
+    TSP_ERR_WORKSPACE = 6          /* workspace NULL or smaller than tsp_mlp_workspace_size */
+} tsp_status_t;
+
+typedef enum {
+    TSP_ACT_GELU = 0,  /* exact erf GeLU: z * (1 + erf(z / sqrt 2)) / 2 */
+    TSP_ACT_SWIGLU = 1 /* SiLU(g) * u with SiLU(g) = g / (1 + exp(-g)) */
+} tsp_act_t;
+
+typedef enum { TSP_DT_BF16 = 0, TSP_DT_F32 = 1 } tsp_dtype_t;
+
+typedef enum {
+    /* Weight-shard schedule: every token meets shard 0, 1, ..., P-1 in order
+     * and the partial outputs accumulate in that order. */
+    TSP_SCHED_WEIGHT_SHARDS = 0,
+    /* Folded tensor-and-sequence ring: tokens form P equal sequence shards;
+     * at ring step t sequence shard s meets weight shard (s + t) mod P.
+     * Needs n % P == 0. */
+    TSP_SCHED_TSP_RING = 1
+} tsp_sched_t;
+
+/* Forward pass, bf16, weight-shard schedule.
+ *   X        [n_tokens][d_model] bf16
+ *   W_gate   [d_model][d_ff] bf16 -- A for TSP_ACT_GELU
+ *   W_up     [d_model][d_ff] bf16 -- must be NULL for TSP_ACT_GELU
+ *   W_down   [d_ff][d_model] bf16 -- B for TSP_ACT_GELU
+ *   Y        [n_tokens][d_model] bf16, written (must not overlap any input)
+ * Requirements: n_tokens, d_model, d_ff > 0; 1 <= P <= 4096; d_ff % P == 0;
+ * d_model % 8 == 0 and (d_ff / P) % 8 == 0 (16-byte rows for TMA);
+ * every pointer 16-byte aligned.  Scratch: cudaMallocAsync on `stream`. */
+TSP_API tsp_status_t tsp_mlp_forward(const void* X, const void* W_gate, const void* W_up,
+                             const void* W_down, int64_t n_tokens, int64_t d_model,
+                             int64_t d_ff, int P, tsp_act_t act, void* Y, tsp_stream_t stream);
+
+/* Forward pass with every option and a caller workspace.
+ *   dtype      TSP_DT_BF16 (tensor cores) or TSP_DT_F32 (fp32 FMA; any sizes)
+ *   sched      TSP_SCHED_WEIGHT_SHARDS or TSP_SCHED_TSP_RING (needs n % P == 0)
+ *   workspace  256-byte aligned device buffer, not overlapping any argument.
+ *              tsp_mlp_workspace_size() gives the preferred size.  For bf16 a
+ *              smaller workspace is accepted: the schedule then uses narrower
+ *              hidden chunks (or fewer sequence shards per ring launch), i.e.
+ *              more passes over the fp32 accumulator, down to one 128-column
+ *              chunk (one sequence shard) plus the [n][d_model] fp32
+ *              accumulator; below that the call returns TSP_ERR_WORKSPACE.
+ *              fp32 needs the preferred size.
+ * Other arguments as tsp_mlp_forward. */
+TSP_API tsp_status_t tsp_mlp_forward_ex(const void* X, const void* W_gate, const void* W_up,
+                                const void* W_down, int64_t n_tokens, int64_t d_model,
+                                int64_t d_ff, int P, tsp_act_t act, tsp_dtype_t dtype,
+                                tsp_sched_t sched, void* Y, void* workspace,
+                                size_t workspace_bytes, tsp_stream_t stream);
+
+/* Backward pass, bf16, weight-shard schedule, for upstream gradient dY.
+ *   dY        [n_tokens][d_model] bf16
+ *   dX        [n_tokens][d_model] bf16, written
+ *   dW_gate   [d_model][d_ff] fp32, written (dA for TSP_ACT_GELU)
+ *   dW_up     [d_model][d_ff] fp32, written; NULL for TSP_ACT_GELU
+ *   dW_down   [d_ff][d_model] fp32, written (dB for TSP_ACT_GELU)
+ * The hidden activations are recomputed from X (no forward state is kept).
+ * Requirements as tsp_mlp_forward; outputs must not overlap inputs or each
+ * other.  Scratch: cudaMallocAsync on `stream`. */
+TSP_API tsp_status_t tsp_mlp_backward(const void* X, const void* W_gate, const void* W_up,
+                              const void* W_down, const void* dY, int64_t n_tokens,
+                              int64_t d_model, int64_t d_ff, int P, tsp_act_t act, void* dX,
+                              float* dW_gate, float* dW_up, float* dW_down,
+                              tsp_stream_t stream);
+
+/* Backward with a caller workspace (bf16 only; weight-shard schedule).  As for
+ * tsp_mlp_forward_ex, a workspace smaller than the preferred size is accepted
+ * down to one 128-column chunk of the hidden buffers plus the fp32 dX
+ * accumulator. */
+TSP_API tsp_status_t tsp_mlp_backward_ex(const void* X, const void* W_gate, const void* W_up,
+                                 const void* W_down, const void* dY, int64_t n_tokens,
+                                 int64_t d_model, int64_t d_ff, int P, tsp_act_t act, void* dX,
+                                 float* dW_gate, float* dW_up, float* dW_down, void* workspace,
+                                 size_t workspace_bytes, tsp_stream_t stream);
+
+/* Preferred bytes of workspace of the _ex calls for these arguments (backward
+ * != 0 for tsp_mlp_backward_ex): hidden chunks sized to stay resident in L2.
+ * Writes *bytes; no device is touched. */
+TSP_API tsp_status_t tsp_mlp_workspace_size(int64_t n_tokens, int64_t d_model, int64_t d_ff, int P,
+                                    tsp_act_t act, tsp_dtype_t dtype, tsp_sched_t sched,
+                                    int backward, size_t* bytes);
+
+/* A static, human-readable name for a status. */
+TSP_API const char* tsp_status_string(tsp_status_t status);
+
+/* Per-kernel tracing.  While enabled, every kernel the library launches is
+ * bracketed by two CUDA events recorded on the stream it is launched on; the
+ * events are kept until tsp_trace_collect().  Process-wide; off by default. */
+typedef struct {
+    const char* name;  /* static string, e.g. "fwd_hidden_swiglu" */
+    int64_t launches;  /* launches since the last reset */
+    double total_ms;   /* sum of their event-timed durations */
+} tsp_kernel_stat_t;
+
+TSP_API tsp_status_t tsp_trace_enable(int enable);
+
+/* Waits for every traced launch to finish, folds them into per-kernel totals
+ * and copies up to `capacity` entries to `stats` (`*count` = entries filled).
+ * Totals accumulate until tsp_trace_reset(). */
+TSP_API tsp_status_t tsp_trace_collect(tsp_kernel_stat_t* stats, int capacity, int* count);
+
+/* Drops all totals and pending events. */
+TSP_API tsp_status_t tsp_trace_reset(void);
+
+/* Synchronises `stream`, then reads and clears the current device's error
+ * word: TSP_OK, TSP_ERR_TIMEOUT if a kernel gave up waiting, TSP_ERR_CUDA if
+ * the stream reported an error. */
+TSP_API tsp_status_t tsp_poll_device_error(tsp_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TSPMLP_H */

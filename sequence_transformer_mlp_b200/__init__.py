@@ -1,0 +1,228 @@
+"""Python binding of libtspmlp, the column-then-row sharded transformer MLP on
+one B200 (sm_100a).
+
+Argument marshalling only: every function below forwards to the C entry
+point of the same name in ``libtspmlp.so`` (declared in ``include/tspmlp.h``),
+and every step of the computation runs in the library's CUDA kernels.  There
+is no CPU fallback: if the library is missing, importing a function raises.
+PyTorch is used only for device memory and streams (``mlp_forward`` and
+``mlp_backward`` allocate outputs and workspace with it).
+
+Arguments that are device buffers accept a ``torch.Tensor`` (its
+``data_ptr()`` is passed) or a plain integer address.  ``stream`` defaults to
+the current torch CUDA stream.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtspmlp.so")
+
+TSP_OK = 0
+STATUS_NAMES = {
+    0: "TSP_OK",
+    1: "TSP_ERR_INVALID_ARG",
+    2: "TSP_ERR_UNSUPPORTED_SHAPE",
+    3: "TSP_ERR_ARCH",
+    4: "TSP_ERR_CUDA",
+    5: "TSP_ERR_TIMEOUT",
+    6: "TSP_ERR_WORKSPACE",
+}
+ACT = {"gelu": 0, "swiglu": 1}
+DTYPE = {"bf16": 0, "f32": 1}
+SCHED = {"weight_shards": 0, "tsp_ring": 1}
+
+
+class KernelStat(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char_p), ("launches", ctypes.c_int64),
+                ("total_ms", ctypes.c_double)]
+
+
+class TspError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+
+
+_lib = None
+
+
+def load(path: str | None = None) -> ctypes.CDLL:
+    """Load libtspmlp.so (built by ``python -m sequence_transformer_mlp_b200.build``)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise ImportError(f"libtspmlp.so not found at {p}; build it with "
+                          "`python -m sequence_transformer_mlp_b200.build`")
+    lib = ctypes.CDLL(p)
+    vp, i64, ci, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+    lib.tsp_mlp_forward.argtypes = [vp, vp, vp, vp, i64, i64, i64, ci, ci, vp, vp]
+    lib.tsp_mlp_forward_ex.argtypes = [vp, vp, vp, vp, i64, i64, i64, ci, ci, ci, ci, vp, vp, sz,
+                                       vp]
+    lib.tsp_mlp_backward.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, ci, ci, vp, vp, vp, vp,
+                                     vp]
+    lib.tsp_mlp_backward_ex.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, ci, ci, vp, vp, vp,
+                                        vp, vp, sz, vp]
+    lib.tsp_mlp_workspace_size.argtypes = [i64, i64, i64, ci, ci, ci, ci, ci,
+                                           ctypes.POINTER(ctypes.c_size_t)]
+    lib.tsp_status_string.argtypes = [ci]
+    lib.tsp_status_string.restype = ctypes.c_char_p
+    lib.tsp_poll_device_error.argtypes = [vp]
+    lib.tsp_trace_enable.argtypes = [ci]
+    lib.tsp_trace_collect.argtypes = [ctypes.POINTER(KernelStat), ci, ctypes.POINTER(ci)]
+    lib.tsp_trace_reset.argtypes = []
+    for name in ("tsp_mlp_forward", "tsp_mlp_forward_ex", "tsp_mlp_backward",
+                 "tsp_mlp_backward_ex", "tsp_mlp_workspace_size", "tsp_poll_device_error",
+                 "tsp_trace_enable", "tsp_trace_collect", "tsp_trace_reset"):
+        getattr(lib, name).restype = ci
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def _addr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _enum(table, v):
+    return table[v] if isinstance(v, str) else int(v)
+
+
+def _check(status: int, where: str) -> None:
+    if status != TSP_OK:
+        raise TspError(status, where)
+
+
+# --------------------------------------------------------------------------- C entry points
+
+
+def tsp_mlp_forward(X, W_gate, W_up, W_down, n_tokens, d_model, d_ff, P, act, Y, stream=None,
+                    check=True) -> int:
+    s = load().tsp_mlp_forward(_addr(X), _addr(W_gate), _addr(W_up), _addr(W_down), n_tokens,
+                               d_model, d_ff, P, _enum(ACT, act), _addr(Y), _stream(stream))
+    if check:
+        _check(s, "tsp_mlp_forward")
+    return s
+
+
+def tsp_mlp_forward_ex(X, W_gate, W_up, W_down, n_tokens, d_model, d_ff, P, act, dtype, sched, Y,
+                       workspace, workspace_bytes, stream=None, check=True) -> int:
+    s = load().tsp_mlp_forward_ex(_addr(X), _addr(W_gate), _addr(W_up), _addr(W_down), n_tokens,
+                                  d_model, d_ff, P, _enum(ACT, act), _enum(DTYPE, dtype),
+                                  _enum(SCHED, sched), _addr(Y), _addr(workspace),
+                                  workspace_bytes, _stream(stream))
+    if check:
+        _check(s, "tsp_mlp_forward_ex")
+    return s
+
+
+def tsp_mlp_backward(X, W_gate, W_up, W_down, dY, n_tokens, d_model, d_ff, P, act, dX, dW_gate,
+                     dW_up, dW_down, stream=None, check=True) -> int:
+    s = load().tsp_mlp_backward(_addr(X), _addr(W_gate), _addr(W_up), _addr(W_down), _addr(dY),
+                                n_tokens, d_model, d_ff, P, _enum(ACT, act), _addr(dX),
+                                _addr(dW_gate), _addr(dW_up), _addr(dW_down), _stream(stream))
+    if check:
+        _check(s, "tsp_mlp_backward")
+    return s
+
+
+def tsp_mlp_backward_ex(X, W_gate, W_up, W_down, dY, n_tokens, d_model, d_ff, P, act, dX, dW_gate,
+                        dW_up, dW_down, workspace, workspace_bytes, stream=None,
+                        check=True) -> int:
+    s = load().tsp_mlp_backward_ex(_addr(X), _addr(W_gate), _addr(W_up), _addr(W_down),
+                                   _addr(dY), n_tokens, d_model, d_ff, P, _enum(ACT, act),
+                                   _addr(dX), _addr(dW_gate), _addr(dW_up), _addr(dW_down),
+                                   _addr(workspace), workspace_bytes, _stream(stream))
+    if check:
+        _check(s, "tsp_mlp_backward_ex")
+    return s
+
+
+def tsp_mlp_workspace_size(n_tokens, d_model, d_ff, P, act, dtype="bf16", sched="weight_shards",
+                           backward=False) -> int:
+    out = ctypes.c_size_t(0)
+    s = load().tsp_mlp_workspace_size(n_tokens, d_model, d_ff, P, _enum(ACT, act),
+                                      _enum(DTYPE, dtype), _enum(SCHED, sched),
+                                      1 if backward else 0, ctypes.byref(out))
+    _check(s, "tsp_mlp_workspace_size")
+    return int(out.value)
+
+
+def tsp_status_string(status: int) -> str:
+    return load().tsp_status_string(int(status)).decode()
+
+
+def tsp_poll_device_error(stream=None) -> int:
+    return int(load().tsp_poll_device_error(_stream(stream)))
+
+
+def tsp_trace_enable(enable: bool = True) -> None:
+    _check(load().tsp_trace_enable(1 if enable else 0), "tsp_trace_enable")
+
+
+def tsp_trace_collect(capacity: int = 64) -> dict:
+    """{kernel name: (launches, total_ms)} accumulated since the last reset."""
+    arr = (KernelStat * capacity)()
+    cnt = ctypes.c_int(0)
+    _check(load().tsp_trace_collect(arr, capacity, ctypes.byref(cnt)), "tsp_trace_collect")
+    return {arr[i].name.decode(): (int(arr[i].launches), float(arr[i].total_ms))
+            for i in range(cnt.value)}
+
+
+def tsp_trace_reset() -> None:
+    _check(load().tsp_trace_reset(), "tsp_trace_reset")
+
+
+# --------------------------------------------------------------------------- torch conveniences
+
+
+def mlp_forward(X, W_gate, W_up, W_down, P: int, act: str, sched: str = "weight_shards",
+                out=None, workspace=None, stream=None):
+    """Y = act-MLP(X) through tsp_mlp_forward_ex; dtype follows X (bf16 or fp32).
+    Allocates Y and the workspace with torch unless given."""
+    import torch
+    n, d = X.shape
+    f = W_gate.shape[1]
+    dt = "bf16" if X.dtype == torch.bfloat16 else "f32"
+    Y = out if out is not None else torch.empty((n, d), dtype=X.dtype, device=X.device)
+    need = tsp_mlp_workspace_size(n, d, f, P, act, dt, sched)
+    ws = workspace
+    if ws is None and need:
+        ws = torch.empty(need, dtype=torch.uint8, device=X.device)
+    tsp_mlp_forward_ex(X, W_gate, W_up, W_down, n, d, f, P, act, dt, sched, Y, ws, need, stream)
+    return Y
+
+
+def mlp_backward(X, W_gate, W_up, W_down, dY, P: int, act: str, workspace=None, stream=None):
+    """(dX bf16, dW_gate fp32, dW_up fp32 or None, dW_down fp32) through
+    tsp_mlp_backward_ex."""
+    import torch
+    n, d = X.shape
+    f = W_gate.shape[1]
+    dev = X.device
+    dX = torch.empty((n, d), dtype=torch.bfloat16, device=dev)
+    dWg = torch.empty((d, f), dtype=torch.float32, device=dev)
+    dWu = torch.empty((d, f), dtype=torch.float32, device=dev) if act == "swiglu" else None
+    dWd = torch.empty((f, d), dtype=torch.float32, device=dev)
+    need = tsp_mlp_workspace_size(n, d, f, P, act, "bf16", "weight_shards", backward=True)
+    ws = workspace if workspace is not None else torch.empty(need, dtype=torch.uint8, device=dev)
+    tsp_mlp_backward_ex(X, W_gate, W_up, W_down, dY, n, d, f, P, act, dX, dWg, dWu, dWd, ws, need,
+                        stream)
+    return dX, dWg, dWu, dWd

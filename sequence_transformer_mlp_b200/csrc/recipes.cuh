@@ -1,0 +1,564 @@
+// recipes.cuh -- the tile recipes run by the tcgen05 pipeline (pipeline.cuh).
+//
+// Shapes: UMMA M = 128 (tile rows = tokens, or weight rows for the weight
+// gradients), N = 128 or 256, K = 16 per instruction; bf16 operands, fp32
+// accumulators in tensor memory.  Operand tiles are staged by TMA with the
+// 128-byte swizzle (64-byte for the K = 32 stages of the backward kernel):
+//   K-major operand, BK = 64: one box {64 k, rows}; 8-row groups 1024 B apart
+//       (SBO); the K = 16 sub-steps advance the start address by 32 B.
+//   K-major operand, BK = 32: one box {32 k, rows} with the 64-byte swizzle;
+//       8-row groups 512 B apart; sub-steps advance by 32 B.
+//   MN-major operand: boxes {64 mn, BK k} side by side; a box is BK rows of
+//       128 B, 8-row groups 1024 B apart (SBO), neighbouring 64-wide MN blocks
+//       BK*128 B apart (LBO); the K = 16 sub-steps advance by 2048 B.
+//
+// Row segments (SegGeom) let one launch cover several independent row blocks,
+// each paired with its own weight shard: the weight-shard schedule uses one
+// segment of all tokens; the folded tensor-and-sequence ring uses one segment
+// per sequence shard, segment s meeting weight shard (s + t) mod P at ring
+// step t ("Folding Tensor and Sequence Parallelism for Memory-Efficient
+// Transformer Training & Inference", Abstract).
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "pipeline.cuh"
+
+namespace tspmlp {
+
+struct SegGeom {
+    int seg_rows;   // rows per segment
+    int num_segs;   // segments in this launch
+    int seg_begin;  // global index of the launch's first segment
+    int ring;       // 1: segment sg uses weight shard (sg + ring_step) mod P
+    int ring_step;
+    int P;
+    int fs;         // hidden columns per weight shard
+    int col_base;   // hidden column base when ring == 0
+    __host__ __device__ __forceinline__ int mtiles() const { return (seg_rows + 127) >> 7; }
+    __host__ __device__ __forceinline__ int shard_col(int s) const {
+        return ring ? ((seg_begin + s + ring_step) % P) * fs : col_base;
+    }
+};
+
+// ----------------------------------------------------------------------------
+// epilogue helpers (one thread = one tile row)
+
+__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
+
+__device__ __forceinline__ float gelu_f(float z) {
+    return 0.5f * z * (1.0f + erff(z * 0.70710678118654752440f));
+}
+
+// 32 bf16 (16 packed words) to dst[0..valid), vectorised when the whole run fits.
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const uint32_t (&pk)[16],
+                                              int valid) {
+    if (valid >= 32) {
+        uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+    } else {
+        uint16_t* d16 = reinterpret_cast<uint16_t*>(dst);
+        for (int i = 0; i < valid; ++i)
+            d16[i] = static_cast<uint16_t>((i & 1) ? (pk[i >> 1] >> 16) : (pk[i >> 1] & 0xFFFFu));
+    }
+}
+
+__device__ __forceinline__ void store_f32x32(float* dst, const uint32_t (&v)[32], int valid) {
+    if (valid >= 32) {
+        float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            d4[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+    } else {
+        for (int i = 0; i < valid; ++i) dst[i] = __uint_as_float(v[i]);
+    }
+}
+
+// ============================================================================
+// K1: column-split gate/up projection with the activation fused.
+//   SwiGLU: H[:, j] = SiLU(X.W_gate[:, c+j]) * (X.W_up[:, c+j]), 128 columns a
+//           tile; one N = 256 UMMA per K-step computes gate (TMEM columns
+//           0-127) and up (128-255) from the same X tile.
+//   GeLU:   H[:, j] = GeLU(X.A[:, c+j]), 256 columns a tile.
+// "Tensor Parallelism: Splitting the Math", steps 2-3: each shard's hidden
+// columns need only X and its own columns of A.
+template <int ACT>  // 0 = GeLU, 1 = SwiGLU
+struct FwdHidden {
+    struct Params {
+        CUtensorMap tmX;  // X [n][d], box {64, 128}
+        CUtensorMap tmG;  // W_gate / A [d][f], box {64, 64}
+        CUtensorMap tmU;  // W_up [d][f], box {64, 64} (SwiGLU)
+        SegGeom g;
+        int d;            // contraction (d_model)
+        int width;        // hidden columns per segment in this launch
+        __nv_bfloat16* H; // [num_segs * seg_rows][width]
+        long long ldh;
+    };
+    static constexpr const char* kName = ACT == 1 ? "fwd_hidden_swiglu" : "fwd_hidden_gelu";
+    static constexpr int kBK = 64;
+    static constexpr int kOut = ACT == 1 ? 128 : 256;
+    static constexpr int kABytes = 128 * kBK * 2;
+    static constexpr int kBBytes = 256 * kBK * 2;
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kStages = 4;
+    static constexpr int kAccCols = 256, kAccBufs = 2, kTmemCols = 512;
+    static constexpr uint32_t kIdesc = make_idesc_bf16(128, 256, false, true);
+    struct Tile {
+        int s, mi, nj;
+    };
+    __host__ __device__ static int num_tiles(const Params& p) {
+        return p.g.num_segs * p.g.mtiles() * ((p.width + kOut - 1) / kOut);
+    }
+    __device__ static Tile tile(const Params& p, int t) {
+        const int mt = p.g.mtiles(), tm = p.g.num_segs * mt;
+        const int m = t % tm;
+        return Tile{m / mt, m % mt, t / tm};
+    }
+    __device__ static int num_kb(const Params& p, const Tile&) { return (p.d + kBK - 1) / kBK; }
+    __device__ static void prefetch(const Params& p) {
+        tma_prefetch_desc(&p.tmX);
+        tma_prefetch_desc(&p.tmG);
+        if (ACT == 1) tma_prefetch_desc(&p.tmU);
+    }
+    __device__ static uint32_t load_bytes(const Params&, const Tile&, int) { return kStageBytes; }
+    __device__ static void load(const Params& p, const Tile& ti, int kb, uint32_t st, uint32_t bar) {
+        const int k0 = kb * kBK;
+        tma_load_2d(st, &p.tmX, bar, k0, (p.g.seg_begin + ti.s) * p.g.seg_rows + ti.mi * 128);
+        const int c = p.g.shard_col(ti.s) + ti.nj * kOut;
+        const uint32_t b = st + kABytes;
+        if (ACT == 1) {
+            tma_load_2d(b, &p.tmG, bar, c, k0);
+            tma_load_2d(b + 8192, &p.tmG, bar, c + 64, k0);
+            tma_load_2d(b + 16384, &p.tmU, bar, c, k0);
+            tma_load_2d(b + 24576, &p.tmU, bar, c + 64, k0);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) tma_load_2d(b + 8192 * i, &p.tmG, bar, c + 64 * i, k0);
+        }
+    }
+    __device__ static void mma(const Tile&, int kb, uint32_t st, uint32_t acc) {
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t a = make_smem_desc(st + 32 * kk, 16, 1024, kLayoutSW128);
+            const uint64_t b = make_smem_desc(st + kABytes + 2048 * kk, 8192, 1024, kLayoutSW128);
+            umma_bf16(acc, a, b, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+        }
+    }
+    __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t acc, int q, int lane) {
+        const int rl = ti.mi * 128 + q * 32 + lane;
+        const bool row_ok = rl < p.g.seg_rows;
+        __nv_bfloat16* hrow = p.H + static_cast<long long>(ti.s * p.g.seg_rows + rl) * p.ldh;
+        const uint32_t t0 = acc + (static_cast<uint32_t>(q * 32) << 16);
+        if (ACT == 1) {
+#pragma unroll 1
+            for (int cc = 0; cc < 4; ++cc) {
+                uint32_t g[32], u[32], pk[16];
+                tmem_ld_32x32b_x32(t0 + 32 * cc, g);
+                tmem_ld_32x32b_x32(t0 + 128 + 32 * cc, u);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float h0 = silu_f(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]);
+                    const float h1 =
+                        silu_f(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
+                    pk[i] = pack_bf16x2(h0, h1);
+                }
+                const int c0 = ti.nj * 128 + 32 * cc;
+                if (row_ok) store_bf16x32(hrow + c0, pk, p.width - c0);
+            }
+        } else {
+#pragma unroll 1
+            for (int cc = 0; cc < 8; ++cc) {
+                uint32_t z[32], pk[16];
+                tmem_ld_32x32b_x32(t0 + 32 * cc, z);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    pk[i] = pack_bf16x2(gelu_f(__uint_as_float(z[2 * i])),
+                                        gelu_f(__uint_as_float(z[2 * i + 1])));
+                const int c0 = ti.nj * 256 + 32 * cc;
+                if (row_ok) store_bf16x32(hrow + c0, pk, p.width - c0);
+            }
+        }
+    }
+};
+
+// ============================================================================
+// K2 / K5: row-split down projection with the partial output added into an
+// fp32 accumulator in place ("Tensor Parallelism: Splitting the Math", steps
+// 4-6: B split by rows to match A's columns, partial outputs summed -- here a
+// local read-modify-write in shard order instead of an all-reduce).
+//   out[rows][0..n_out) (+)= sum over K-segments of A_seg . B_seg
+// A is K-major (hidden activations, [rows][kdim]); B is MN-major (W_down
+// [f][d], forward) or K-major (W_gate / W_up [d][f], input gradient).
+// Modes: 0 store fp32, 1 add into fp32, 2 bf16(acc + tile) to out, 3 bf16(tile).
+template <bool B_MN, int NSEG>
+struct DownAccum {
+    struct Params {
+        CUtensorMap tmA0, tmB0, tmA1, tmB1;
+        SegGeom g;        // shard_col(s): hidden index base of segment s in B
+        int kdim;         // hidden columns per K-segment
+        int n_out;        // output columns
+        int mode;
+        float* acc;       // [rows][n_out] fp32 accumulator (global rows)
+        long long ldacc;
+        __nv_bfloat16* out;  // [rows][n_out] bf16 (global rows)
+        long long ldo;
+    };
+    static constexpr const char* kName =
+        B_MN ? "down_accum_fwd" : (NSEG == 2 ? "dgrad_accum_swiglu" : "dgrad_accum_gelu");
+    static constexpr int kBK = 64;
+    static constexpr int kABytes = 128 * kBK * 2;
+    static constexpr int kBBytes = 256 * kBK * 2;
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kStages = 4;
+    static constexpr int kAccCols = 256, kAccBufs = 2, kTmemCols = 512;
+    static constexpr uint32_t kIdesc = make_idesc_bf16(128, 256, false, B_MN);
+    struct Tile {
+        int s, mi, nj;
+    };
+    __host__ __device__ static int num_tiles(const Params& p) {
+        return p.g.num_segs * p.g.mtiles() * ((p.n_out + 255) / 256);
+    }
+    __device__ static Tile tile(const Params& p, int t) {
+        const int mt = p.g.mtiles(), tm = p.g.num_segs * mt;
+        const int m = t % tm;
+        return Tile{m / mt, m % mt, t / tm};
+    }
+    __device__ static int num_kb(const Params& p, const Tile&) {
+        return NSEG * ((p.kdim + kBK - 1) / kBK);
+    }
+    __device__ static void prefetch(const Params& p) {
+        tma_prefetch_desc(&p.tmA0);
+        tma_prefetch_desc(&p.tmB0);
+        if (NSEG > 1) {
+            tma_prefetch_desc(&p.tmA1);
+            tma_prefetch_desc(&p.tmB1);
+        }
+    }
+    __device__ static uint32_t load_bytes(const Params&, const Tile&, int) { return kStageBytes; }
+    __device__ static void load(const Params& p, const Tile& ti, int kb, uint32_t st, uint32_t bar) {
+        const int nkb1 = (p.kdim + kBK - 1) / kBK;
+        const int seg = NSEG > 1 ? kb / nkb1 : 0;
+        const int k = (kb - seg * nkb1) * kBK;
+        const CUtensorMap* ta = seg ? &p.tmA1 : &p.tmA0;
+        const CUtensorMap* tb = seg ? &p.tmB1 : &p.tmB0;
+        tma_load_2d(st, ta, bar, k, ti.s * p.g.seg_rows + ti.mi * 128);
+        const int kbase = p.g.shard_col(ti.s);
+        const uint32_t b = st + kABytes;
+        if (B_MN) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) tma_load_2d(b + 8192 * i, tb, bar, ti.nj * 256 + 64 * i, kbase + k);
+        } else {
+            tma_load_2d(b, tb, bar, kbase + k, ti.nj * 256);
+        }
+    }
+    __device__ static void mma(const Tile&, int kb, uint32_t st, uint32_t acc) {
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t a = make_smem_desc(st + 32 * kk, 16, 1024, kLayoutSW128);
+            const uint64_t b = B_MN ? make_smem_desc(st + kABytes + 2048 * kk, 8192, 1024, kLayoutSW128)
+                                    : make_smem_desc(st + kABytes + 32 * kk, 16, 1024, kLayoutSW128);
+            umma_bf16(acc, a, b, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+        }
+    }
+    __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t acc, int q, int lane) {
+        const int rl = ti.mi * 128 + q * 32 + lane;
+        const bool row_ok = rl < p.g.seg_rows;
+        const long long row = static_cast<long long>(p.g.seg_begin + ti.s) * p.g.seg_rows + rl;
+        const uint32_t t0 = acc + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll 1
+        for (int cc = 0; cc < 8; ++cc) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(t0 + 32 * cc, v);
+            tmem_ld_wait();
+            const int c0 = ti.nj * 256 + 32 * cc;
+            const int valid = p.n_out - c0;
+            if (!row_ok || valid <= 0) continue;
+            if (p.mode == 0) {
+                store_f32x32(p.acc + row * p.ldacc + c0, v, valid);
+            } else if (p.mode == 1) {
+                float* a = p.acc + row * p.ldacc + c0;
+                if (valid >= 32) {
+                    float4* a4 = reinterpret_cast<float4*>(a);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        float4 o = a4[i];
+                        o.x += __uint_as_float(v[4 * i]);
+                        o.y += __uint_as_float(v[4 * i + 1]);
+                        o.z += __uint_as_float(v[4 * i + 2]);
+                        o.w += __uint_as_float(v[4 * i + 3]);
+                        a4[i] = o;
+                    }
+                } else {
+                    for (int i = 0; i < valid; ++i) a[i] += __uint_as_float(v[i]);
+                }
+            } else {
+                uint32_t pk[16];
+                if (p.mode == 2) {
+                    const float* a = p.acc + row * p.ldacc + c0;
+                    if (valid >= 32) {
+                        const float4* a4 = reinterpret_cast<const float4*>(a);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const float4 o = a4[i];
+                            pk[2 * i] = pack_bf16x2(o.x + __uint_as_float(v[4 * i]),
+                                                    o.y + __uint_as_float(v[4 * i + 1]));
+                            pk[2 * i + 1] = pack_bf16x2(o.z + __uint_as_float(v[4 * i + 2]),
+                                                        o.w + __uint_as_float(v[4 * i + 3]));
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const float x0 = (2 * i < valid ? a[2 * i] : 0.f) + __uint_as_float(v[2 * i]);
+                            const float x1 = (2 * i + 1 < valid ? a[2 * i + 1] : 0.f) +
+                                             __uint_as_float(v[2 * i + 1]);
+                            pk[i] = pack_bf16x2(x0, x1);
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+                }
+                store_bf16x32(p.out + row * p.ldo + c0, pk, valid);
+            }
+        }
+    }
+};
+
+// ============================================================================
+// K3: backward of the hidden layer for one column chunk.  Per tile (128 tokens
+// x 128 hidden columns) one pipeline computes, over K = d_model,
+//   G = X.W_gate[:, c..]  (and U = X.W_up[:, c..])   -- the recomputed forward
+//   dH = dY.W_down[c.., :]^T
+// and the epilogue emits H (for the W_down gradient) and the pre-activation
+// gradients: SwiGLU dU = dH SiLU(G), dG = dH U SiLU'(G); GeLU dG = dH GeLU'(G).
+// The pages only say the backward repeats the forward's pattern
+// ("Tensor Parallelism: Splitting the Math", the traffic count); the
+// derivatives are those of the forward definition.
+template <int ACT>
+struct BwdHidden {
+    struct Params {
+        CUtensorMap tmX;   // X  [n][d], box {32, 128}, 64B swizzle
+        CUtensorMap tmDY;  // dY [n][d], box {32, 128}, 64B swizzle
+        CUtensorMap tmG;   // W_gate / A [d][f], box {64, 32}
+        CUtensorMap tmU;   // W_up [d][f], box {64, 32} (SwiGLU)
+        CUtensorMap tmD;   // W_down / B [f][d], box {32, 128}, 64B swizzle
+        int n, d, col_base, width;
+        __nv_bfloat16 *H, *dG, *dU;  // [n][width]
+        long long ld;
+    };
+    static constexpr const char* kName = ACT == 1 ? "bwd_hidden_swiglu" : "bwd_hidden_gelu";
+    static constexpr int kBK = 32;
+    static constexpr int kTile = 8192;  // one 128 x 32 bf16 box
+    static constexpr int kOffX = 0, kOffDY = kTile, kOffG = 2 * kTile;
+    static constexpr int kOffU = 3 * kTile;
+    static constexpr int kOffD = ACT == 1 ? 4 * kTile : 3 * kTile;
+    static constexpr int kStageBytes = kOffD + kTile;
+    static constexpr int kStages = ACT == 1 ? 5 : 6;
+    static constexpr int kNGate = ACT == 1 ? 256 : 128;
+    static constexpr int kAccCols = ACT == 1 ? 512 : 256;
+    static constexpr int kAccBufs = ACT == 1 ? 1 : 2;
+    static constexpr int kTmemCols = 512;
+    static constexpr int kColDH = kNGate;  // TMEM column of dH
+    static constexpr uint32_t kIdesc1 = make_idesc_bf16(128, kNGate, false, true);
+    static constexpr uint32_t kIdesc2 = make_idesc_bf16(128, 128, false, false);
+    struct Tile {
+        int mi, nj;
+    };
+    __host__ __device__ static int num_tiles(const Params& p) {
+        return ((p.n + 127) / 128) * ((p.width + 127) / 128);
+    }
+    __device__ static Tile tile(const Params& p, int t) {
+        const int mt = (p.n + 127) / 128;
+        return Tile{t % mt, t / mt};
+    }
+    __device__ static int num_kb(const Params& p, const Tile&) { return (p.d + kBK - 1) / kBK; }
+    __device__ static void prefetch(const Params& p) {
+        tma_prefetch_desc(&p.tmX);
+        tma_prefetch_desc(&p.tmDY);
+        tma_prefetch_desc(&p.tmG);
+        if (ACT == 1) tma_prefetch_desc(&p.tmU);
+        tma_prefetch_desc(&p.tmD);
+    }
+    __device__ static uint32_t load_bytes(const Params&, const Tile&, int) { return kStageBytes; }
+    __device__ static void load(const Params& p, const Tile& ti, int kb, uint32_t st, uint32_t bar) {
+        const int k0 = kb * kBK;
+        const int r = ti.mi * 128;
+        const int c = p.col_base + ti.nj * 128;
+        tma_load_2d(st + kOffX, &p.tmX, bar, k0, r);
+        tma_load_2d(st + kOffDY, &p.tmDY, bar, k0, r);
+        tma_load_2d(st + kOffG, &p.tmG, bar, c, k0);
+        tma_load_2d(st + kOffG + 4096, &p.tmG, bar, c + 64, k0);
+        if (ACT == 1) {
+            tma_load_2d(st + kOffU, &p.tmU, bar, c, k0);
+            tma_load_2d(st + kOffU + 4096, &p.tmU, bar, c + 64, k0);
+        }
+        tma_load_2d(st + kOffD, &p.tmD, bar, k0, c);
+    }
+    __device__ static void mma(const Tile&, int kb, uint32_t st, uint32_t acc) {
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint32_t en = (kb | kk) != 0 ? 1u : 0u;
+            const uint64_t ax = make_smem_desc(st + kOffX + 32 * kk, 16, 512, kLayoutSW64);
+            const uint64_t bg = make_smem_desc(st + kOffG + 2048 * kk, 4096, 1024, kLayoutSW128);
+            umma_bf16(acc, ax, bg, kIdesc1, en);
+            const uint64_t ady = make_smem_desc(st + kOffDY + 32 * kk, 16, 512, kLayoutSW64);
+            const uint64_t bd = make_smem_desc(st + kOffD + 32 * kk, 16, 512, kLayoutSW64);
+            umma_bf16(acc + kColDH, ady, bd, kIdesc2, en);
+        }
+    }
+    __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t acc, int q, int lane) {
+        const int row = ti.mi * 128 + q * 32 + lane;
+        const bool row_ok = row < p.n;
+        const long long off = static_cast<long long>(row) * p.ld;
+        const uint32_t t0 = acc + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+            uint32_t g[32], dh[32], ph[16], pg[16], pu[16];
+            tmem_ld_32x32b_x32(t0 + 32 * cc, g);
+            tmem_ld_32x32b_x32(t0 + kColDH + 32 * cc, dh);
+            if (ACT == 1) {
+                uint32_t u[32];
+                tmem_ld_32x32b_x32(t0 + 128 + 32 * cc, u);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    float hh[2], gg[2], uu[2];
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const float gv = __uint_as_float(g[2 * i + j]);
+                        const float uv = __uint_as_float(u[2 * i + j]);
+                        const float dv = __uint_as_float(dh[2 * i + j]);
+                        const float sg = 1.0f / (1.0f + __expf(-gv));
+                        const float si = gv * sg;
+                        hh[j] = si * uv;
+                        uu[j] = dv * si;
+                        gg[j] = dv * uv * sg * (1.0f + gv * (1.0f - sg));
+                    }
+                    ph[i] = pack_bf16x2(hh[0], hh[1]);
+                    pg[i] = pack_bf16x2(gg[0], gg[1]);
+                    pu[i] = pack_bf16x2(uu[0], uu[1]);
+                }
+            } else {
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    float hh[2], gg[2];
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const float z = __uint_as_float(g[2 * i + j]);
+                        const float dv = __uint_as_float(dh[2 * i + j]);
+                        const float cdf = 0.5f * (1.0f + erff(z * 0.70710678118654752440f));
+                        const float pdf = 0.39894228040143267794f * __expf(-0.5f * z * z);
+                        hh[j] = z * cdf;
+                        gg[j] = dv * (cdf + z * pdf);
+                    }
+                    ph[i] = pack_bf16x2(hh[0], hh[1]);
+                    pg[i] = pack_bf16x2(gg[0], gg[1]);
+                }
+            }
+            const int c0 = ti.nj * 128 + 32 * cc;
+            if (row_ok) {
+                store_bf16x32(p.H + off + c0, ph, p.width - c0);
+                store_bf16x32(p.dG + off + c0, pg, p.width - c0);
+                if (ACT == 1) store_bf16x32(p.dU + off + c0, pu, p.width - c0);
+            }
+        }
+    }
+};
+
+// ============================================================================
+// K4: weight gradients, contraction over tokens.  Both operands MN-major.
+//   out[r][c] = sum_tok A[tok][a_col0 + r] * B[tok][b_col0 + c]
+// SPLIT: B is two 128-column sources (dG | dU) written to out0 | out1
+// (dW_gate, dW_up share the X operand); otherwise one source of NCOLS.
+template <int NCOLS, bool SPLIT>
+struct Wgrad {
+    struct Params {
+        CUtensorMap tmA, tmB0, tmB1;  // [ntok][*] bf16, box {64, 64}
+        int ntok;
+        int m_valid, n_valid;         // rows / columns of the output block
+        int a_col0, b_col0;
+        float* out0;
+        float* out1;
+        long long ldo;
+        int out_row0, out_col0;
+    };
+    static constexpr const char* kName =
+        SPLIT ? "wgrad_gate_up" : (NCOLS == 256 ? "wgrad_down" : "wgrad_gelu_a");
+    static constexpr int kBK = 64;
+    static constexpr int kABytes = 128 * kBK * 2;
+    static constexpr int kBBytes = NCOLS * kBK * 2;
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kStages = kStageBytes <= 32768 ? 6 : 4;
+    static constexpr int kAccCols = 256, kAccBufs = 2, kTmemCols = 512;
+    static constexpr int kTileCols = SPLIT ? NCOLS / 2 : NCOLS;
+    static constexpr uint32_t kIdesc = make_idesc_bf16(128, NCOLS, true, true);
+    struct Tile {
+        int mi, nj;
+    };
+    __host__ __device__ static int num_tiles(const Params& p) {
+        return ((p.m_valid + 127) / 128) * ((p.n_valid + kTileCols - 1) / kTileCols);
+    }
+    __device__ static Tile tile(const Params& p, int t) {
+        const int mt = (p.m_valid + 127) / 128;
+        return Tile{t % mt, t / mt};
+    }
+    __device__ static int num_kb(const Params& p, const Tile&) { return (p.ntok + kBK - 1) / kBK; }
+    __device__ static void prefetch(const Params& p) {
+        tma_prefetch_desc(&p.tmA);
+        tma_prefetch_desc(&p.tmB0);
+        if (SPLIT) tma_prefetch_desc(&p.tmB1);
+    }
+    __device__ static uint32_t load_bytes(const Params&, const Tile&, int) { return kStageBytes; }
+    __device__ static void load(const Params& p, const Tile& ti, int kb, uint32_t st, uint32_t bar) {
+        const int k0 = kb * kBK;
+        const int a = p.a_col0 + ti.mi * 128;
+        tma_load_2d(st, &p.tmA, bar, a, k0);
+        tma_load_2d(st + 8192, &p.tmA, bar, a + 64, k0);
+        const uint32_t b = st + kABytes;
+        if (SPLIT) {
+            const int c = p.b_col0 + ti.nj * (NCOLS / 2);
+#pragma unroll
+            for (int i = 0; i < NCOLS / 128; ++i) {
+                tma_load_2d(b + 8192 * i, &p.tmB0, bar, c + 64 * i, k0);
+                tma_load_2d(b + 8192 * (i + NCOLS / 128), &p.tmB1, bar, c + 64 * i, k0);
+            }
+        } else {
+            const int c = p.b_col0 + ti.nj * NCOLS;
+#pragma unroll
+            for (int i = 0; i < NCOLS / 64; ++i) tma_load_2d(b + 8192 * i, &p.tmB0, bar, c + 64 * i, k0);
+        }
+    }
+    __device__ static void mma(const Tile&, int kb, uint32_t st, uint32_t acc) {
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t a = make_smem_desc(st + 2048 * kk, 8192, 1024, kLayoutSW128);
+            const uint64_t b = make_smem_desc(st + kABytes + 2048 * kk, 8192, 1024, kLayoutSW128);
+            umma_bf16(acc, a, b, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+        }
+    }
+    __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t acc, int q, int lane) {
+        const int rl = ti.mi * 128 + q * 32 + lane;
+        const bool row_ok = rl < p.m_valid;
+        const long long row = static_cast<long long>(p.out_row0 + rl);
+        const uint32_t t0 = acc + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll 1
+        for (int cc = 0; cc < NCOLS / 32; ++cc) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(t0 + 32 * cc, v);
+            tmem_ld_wait();
+            const int which = SPLIT ? cc / (NCOLS / 64) : 0;
+            const int cl = ti.nj * kTileCols + 32 * (SPLIT ? cc % (NCOLS / 64) : cc);
+            float* o = which ? p.out1 : p.out0;
+            if (row_ok) store_f32x32(o + row * p.ldo + p.out_col0 + cl, v, p.n_valid - cl);
+        }
+    }
+};
+
+}  // namespace tspmlp

@@ -1,0 +1,866 @@
+// tspmlp.cu -- the C ABI of libtspmlp (include/tspmlp.h): argument
+// validation, the host schedule builder that turns (n, d_model, d_ff, P,
+// schedule) into kernel launches, TMA descriptor encoding, and the launches.
+//
+// The method: "Tensor Parallelism: Splitting the Math" (column split of A,
+// row split of B, partial outputs summed into the exact result) and "Folding
+// Tensor and Sequence Parallelism for Memory-Efficient Transformer Training &
+// Inference", Abstract (gated MLP; weight shards meet every sequence shard in
+// ring order while partial outputs accumulate locally).  On one GPU the P
+// shards are logical: the schedule visits them in order and adds each
+// partial output into an fp32 accumulator in place.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/tspmlp.h"
+#include "recipes.cuh"
+#include "simt_f32.cuh"
+
+namespace tspmlp {
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+// Scratch budgets: the hidden chunk(s) of one pass should stay resident in the
+// 126 MB L2 between the producing and the consuming kernel.
+constexpr size_t kFwdHiddenBudget = 64ull << 20;   // one bf16 [rows][C] buffer
+constexpr size_t kBwdHiddenBudget = 96ull << 20;   // H, dG, dU together
+
+struct DevInfo {
+    bool probed = false;
+    bool arch_ok = false;
+    int sms = 0;
+};
+
+std::mutex g_mu;
+DevInfo g_dev[kMaxDevices];
+
+tsp_status_t current_device(int* dev_out, DevInfo* info) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return TSP_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return TSP_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DevInfo& di = g_dev[dev];
+    if (!di.probed) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return TSP_ERR_CUDA;
+        di.arch_ok = (major == 10 && minor == 0);
+        di.sms = sms;
+        di.probed = true;
+    }
+    *dev_out = dev;
+    *info = di;
+    return di.arch_ok ? TSP_OK : TSP_ERR_ARCH;
+}
+
+// ---------------------------------------------------------------------------
+// TMA descriptors through the driver entry point (no link against libcuda)
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// Row-major bf16 matrix [outer][inner] with row pitch `pitch` elements, box
+// {box_in, box_out}; out-of-range elements read as zero.
+bool tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t pitch,
+               uint32_t box_in, uint32_t box_out, CUtensorMapSwizzle sw) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {pitch * 2};
+    cuuint32_t box[2] = {box_in, box_out};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+               es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+constexpr CUtensorMapSwizzle SW128 = CU_TENSOR_MAP_SWIZZLE_128B;
+constexpr CUtensorMapSwizzle SW64 = CU_TENSOR_MAP_SWIZZLE_64B;
+
+// ---------------------------------------------------------------------------
+// tracing: CUDA events around each launch, on the launching stream
+
+struct TraceRec {
+    const char* name;
+    cudaEvent_t a, b;
+};
+struct TraceStat {
+    const char* name;
+    int64_t launches;
+    double ms;
+};
+std::mutex g_trace_mu;
+bool g_trace_on = false;
+std::vector<TraceRec> g_trace_pending;
+std::vector<TraceStat> g_trace_stats;
+
+// Records the start event of a traced launch; returns false if tracing is off.
+bool trace_begin(cudaStream_t st, TraceRec* rec, const char* name) {
+    {
+        std::lock_guard<std::mutex> lk(g_trace_mu);
+        if (!g_trace_on) return false;
+    }
+    rec->name = name;
+    if (cudaEventCreate(&rec->a) != cudaSuccess) return false;
+    if (cudaEventCreate(&rec->b) != cudaSuccess) {
+        cudaEventDestroy(rec->a);
+        return false;
+    }
+    cudaEventRecord(rec->a, st);
+    return true;
+}
+
+void trace_end(cudaStream_t st, TraceRec* rec) {
+    cudaEventRecord(rec->b, st);
+    std::lock_guard<std::mutex> lk(g_trace_mu);
+    g_trace_pending.push_back(*rec);
+}
+
+// ---------------------------------------------------------------------------
+// launches
+
+template <class R>
+tsp_status_t launch_umma(const typename R::Params& p, cudaStream_t st, int dev, int sms) {
+    const int tiles = R::num_tiles(p);
+    if (tiles <= 0) return TSP_OK;
+    constexpr int smem = pipeline_smem_bytes<R>();
+    static_assert(smem <= 232448, "stage ring exceeds 227 KB of shared memory");
+    static bool attr_set[kMaxDevices] = {};
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!attr_set[dev]) {
+            if (cudaFuncSetAttribute(umma_pipeline_kernel<R>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     smem) != cudaSuccess)
+                return TSP_ERR_CUDA;
+            attr_set[dev] = true;
+        }
+    }
+    const int grid = std::min(tiles, sms);
+    TraceRec rec;
+    const bool traced = trace_begin(st, &rec, R::kName);
+    umma_pipeline_kernel<R><<<grid, kPipelineThreads, smem, st>>>(p);
+    const cudaError_t e = cudaGetLastError();
+    if (traced) trace_end(st, &rec);
+    return e == cudaSuccess ? TSP_OK : TSP_ERR_CUDA;
+}
+
+#define TSP_TRY(expr)                          \
+    do {                                       \
+        const tsp_status_t _s = (expr);        \
+        if (_s != TSP_OK) return _s;           \
+    } while (0)
+
+// ---------------------------------------------------------------------------
+// schedule builder
+
+struct Chunk {
+    int64_t col_base, width;
+};
+
+// Hidden-column chunks of the weight-shard schedule, in shard order, at most
+// max_cols wide.  A chunk is a run of whole shards (the largest divisor G of P
+// whose G shards fit) or, when one shard alone is too wide, an equal cut of a
+// shard into 128-multiple sub-chunks.  Chunk edges always include the shard
+// edges, so every chunk belongs to one shard or is a union of whole shards.
+std::vector<Chunk> plan_chunks(int64_t f, int P, int64_t max_cols) {
+    const int64_t fs = f / P;
+    std::vector<Chunk> out;
+    if (fs <= max_cols) {
+        int G = 1;
+        for (int g = P; g >= 1; --g)
+            if (P % g == 0 && g * fs <= max_cols) {
+                G = g;
+                break;
+            }
+        for (int w = 0; w < P; w += G) out.push_back({w * fs, G * fs});
+    } else {
+        const int64_t k = (fs + max_cols - 1) / max_cols;
+        const int64_t sub = ((fs + k - 1) / k + 127) / 128 * 128;
+        for (int w = 0; w < P; ++w)
+            for (int64_t c = 0; c < fs; c += sub) out.push_back({w * fs + c, std::min(sub, fs - c)});
+    }
+    return out;
+}
+
+// Widest chunk (a multiple of 128 columns, at least 128) whose hidden buffers
+// fit `budget` bytes at `bytes_per_col` bytes a hidden column; 0 if none.
+int64_t max_chunk_cols(size_t budget, size_t bytes_per_col) {
+    const int64_t c = static_cast<int64_t>(budget / std::max<size_t>(bytes_per_col, 1)) / 128 * 128;
+    return c >= 128 ? c : 0;
+}
+
+inline size_t align256(size_t b) { return (b + 255) / 256 * 256; }
+
+int accum_mode(int pass, int npass) {
+    if (npass == 1) return 3;          // bf16(tile)
+    if (pass == 0) return 0;           // store fp32
+    if (pass == npass - 1) return 2;   // bf16(acc + tile)
+    return 1;                          // acc += tile
+}
+
+// ---------------------------------------------------------------------------
+// validation
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+    if (!a || !b || na == 0 || nb == 0) return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + nb && b0 < a0 + na;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int64_t kMaxDim = int64_t(1) << 30;
+
+tsp_status_t validate_shape(int64_t n, int64_t d, int64_t f, int P, tsp_act_t act,
+                            tsp_dtype_t dt, tsp_sched_t sched) {
+    if (act != TSP_ACT_GELU && act != TSP_ACT_SWIGLU) return TSP_ERR_INVALID_ARG;
+    if (dt != TSP_DT_BF16 && dt != TSP_DT_F32) return TSP_ERR_INVALID_ARG;
+    if (sched != TSP_SCHED_WEIGHT_SHARDS && sched != TSP_SCHED_TSP_RING) return TSP_ERR_INVALID_ARG;
+    if (n <= 0 || d <= 0 || f <= 0 || P <= 0) return TSP_ERR_INVALID_ARG;
+    if (n > kMaxDim || d > kMaxDim || f > kMaxDim || P > 4096) return TSP_ERR_UNSUPPORTED_SHAPE;
+    if (f % P != 0) return TSP_ERR_UNSUPPORTED_SHAPE;
+    if (sched == TSP_SCHED_TSP_RING && n % P != 0) return TSP_ERR_UNSUPPORTED_SHAPE;
+    if (dt == TSP_DT_BF16 && (d % 8 != 0 || (f / P) % 8 != 0)) return TSP_ERR_UNSUPPORTED_SHAPE;
+    return TSP_OK;
+}
+
+tsp_status_t validate_weights(const void* X, const void* Wg, const void* Wu, const void* Wd,
+                              tsp_act_t act) {
+    if (!X || !Wg || !Wd) return TSP_ERR_INVALID_ARG;
+    if ((act == TSP_ACT_GELU) != (Wu == nullptr)) return TSP_ERR_INVALID_ARG;
+    return TSP_OK;
+}
+
+tsp_status_t validate_forward(const void* X, const void* Wg, const void* Wu, const void* Wd,
+                              int64_t n, int64_t d, int64_t f, int P, tsp_act_t act, tsp_dtype_t dt,
+                              tsp_sched_t sched, const void* Y) {
+    TSP_TRY(validate_shape(n, d, f, P, act, dt, sched));
+    TSP_TRY(validate_weights(X, Wg, Wu, Wd, act));
+    if (!Y) return TSP_ERR_INVALID_ARG;
+    const size_t e = dt == TSP_DT_BF16 ? 2 : 4;
+    const size_t xb = n * d * e, wb = d * f * e, yb = n * d * e;
+    if (overlaps(Y, yb, X, xb) || overlaps(Y, yb, Wg, wb) || overlaps(Y, yb, Wu, wb) ||
+        overlaps(Y, yb, Wd, wb))
+        return TSP_ERR_INVALID_ARG;
+    if (dt == TSP_DT_BF16 && (!aligned16(X) || !aligned16(Wg) || !aligned16(Wd) || !aligned16(Y) ||
+                              (Wu && !aligned16(Wu))))
+        return TSP_ERR_UNSUPPORTED_SHAPE;
+    if (dt == TSP_DT_F32) {
+        const void* ps[5] = {X, Wg, Wu, Wd, Y};
+        for (const void* q : ps)
+            if (q && (reinterpret_cast<uintptr_t>(q) & 3u)) return TSP_ERR_UNSUPPORTED_SHAPE;
+    }
+    return TSP_OK;
+}
+
+tsp_status_t validate_backward(const void* X, const void* Wg, const void* Wu, const void* Wd,
+                               const void* dY, int64_t n, int64_t d, int64_t f, int P,
+                               tsp_act_t act, const void* dX, const float* dWg, const float* dWu,
+                               const float* dWd) {
+    TSP_TRY(validate_shape(n, d, f, P, act, TSP_DT_BF16, TSP_SCHED_WEIGHT_SHARDS));
+    TSP_TRY(validate_weights(X, Wg, Wu, Wd, act));
+    if (!dY || !dX || !dWg || !dWd) return TSP_ERR_INVALID_ARG;
+    if ((act == TSP_ACT_SWIGLU) != (dWu != nullptr)) return TSP_ERR_INVALID_ARG;
+    const size_t xb = n * d * 2, wb = d * f * 2, gw = d * f * 4;
+    const void* ins[5] = {X, Wg, Wu, Wd, dY};
+    const size_t insz[5] = {xb, wb, wb, wb, xb};
+    const void* outs[4] = {dX, dWg, dWu, dWd};
+    const size_t outsz[4] = {xb, gw, gw, gw};
+    for (int o = 0; o < 4; ++o) {
+        for (int i = 0; i < 5; ++i)
+            if (overlaps(outs[o], outsz[o], ins[i], insz[i])) return TSP_ERR_INVALID_ARG;
+        for (int o2 = o + 1; o2 < 4; ++o2)
+            if (overlaps(outs[o], outsz[o], outs[o2], outsz[o2])) return TSP_ERR_INVALID_ARG;
+    }
+    for (int i = 0; i < 5; ++i)
+        if (ins[i] && !aligned16(ins[i])) return TSP_ERR_UNSUPPORTED_SHAPE;
+    for (int o = 0; o < 4; ++o)
+        if (outs[o] && !aligned16(outs[o])) return TSP_ERR_UNSUPPORTED_SHAPE;
+    return TSP_OK;
+}
+
+// ---------------------------------------------------------------------------
+// forward
+
+struct FwdPlan {
+    bool ok = true;
+    bool ring = false;
+    std::vector<Chunk> chunks;  // weight-shard schedule
+    int tsp_group = 1;          // ring schedule: sequence shards per launch
+    size_t h_bytes = 0, acc_bytes = 0;
+    size_t total() const { return align256(h_bytes) + align256(acc_bytes); }
+};
+
+// Schedule of the forward pass for a hidden-buffer budget.  ok == false when
+// not even the narrowest schedule fits.
+FwdPlan plan_forward_budget(int64_t n, int64_t d, int64_t f, int P, tsp_dtype_t dt,
+                            tsp_sched_t sched, size_t budget) {
+    FwdPlan pl;
+    const size_t e = dt == TSP_DT_BF16 ? 2 : 4;
+    const int64_t fs = f / P;
+    if (sched == TSP_SCHED_TSP_RING) {
+        pl.ring = true;
+        const size_t per_seg = static_cast<size_t>(n / P) * fs * e;
+        pl.tsp_group = dt == TSP_DT_BF16
+                           ? static_cast<int>(std::min<size_t>(P, budget / std::max<size_t>(per_seg, 1)))
+                           : P;
+        if (pl.tsp_group < 1) {
+            pl.tsp_group = 1;
+            pl.ok = budget >= per_seg;
+        }
+        pl.h_bytes = static_cast<size_t>(pl.tsp_group) * per_seg;
+        pl.acc_bytes = (dt == TSP_DT_BF16 && P > 1) ? static_cast<size_t>(n) * d * 4 : 0;
+        return pl;
+    }
+    if (dt == TSP_DT_BF16) {
+        const int64_t mc = max_chunk_cols(budget, static_cast<size_t>(n) * 2);
+        if (mc == 0) {
+            pl.ok = false;
+            return pl;
+        }
+        pl.chunks = plan_chunks(f, P, mc);
+    } else {
+        for (int w = 0; w < P; ++w) pl.chunks.push_back({w * fs, fs});
+    }
+    int64_t wmax = 0;
+    for (auto& c : pl.chunks) wmax = std::max(wmax, c.width);
+    pl.h_bytes = static_cast<size_t>(n) * wmax * e;
+    pl.acc_bytes = (dt == TSP_DT_BF16 && pl.chunks.size() > 1) ? static_cast<size_t>(n) * d * 4 : 0;
+    return pl;
+}
+
+// The preferred schedule: hidden buffers within the L2-sized budget.
+FwdPlan plan_forward(int64_t n, int64_t d, int64_t f, int P, tsp_dtype_t dt, tsp_sched_t sched) {
+    return plan_forward_budget(n, d, f, P, dt, sched, kFwdHiddenBudget);
+}
+
+// The schedule for a caller workspace of ws_bytes: the preferred one if it
+// fits, otherwise narrower hidden chunks (bf16 only).
+FwdPlan plan_forward_for(int64_t n, int64_t d, int64_t f, int P, tsp_dtype_t dt, tsp_sched_t sched,
+                         size_t ws_bytes) {
+    FwdPlan pl = plan_forward(n, d, f, P, dt, sched);
+    if (pl.total() <= ws_bytes || dt != TSP_DT_BF16) return pl;
+    const size_t acc = align256(static_cast<size_t>(n) * d * 4);
+    if (ws_bytes <= acc + 256) {
+        pl.ok = false;
+        return pl;
+    }
+    pl = plan_forward_budget(n, d, f, P, dt, sched, ws_bytes - acc - 256);
+    if (pl.total() > ws_bytes) pl.ok = false;
+    return pl;
+}
+
+SegGeom seg_all_rows(int64_t n, int P, int64_t fs, int64_t col_base) {
+    SegGeom g{};
+    g.seg_rows = static_cast<int>(n);
+    g.num_segs = 1;
+    g.seg_begin = 0;
+    g.ring = 0;
+    g.ring_step = 0;
+    g.P = P;
+    g.fs = static_cast<int>(fs);
+    g.col_base = static_cast<int>(col_base);
+    return g;
+}
+
+SegGeom seg_ring(int64_t n, int P, int64_t fs, int seg_begin, int num_segs, int t) {
+    SegGeom g{};
+    g.seg_rows = static_cast<int>(n / P);
+    g.num_segs = num_segs;
+    g.seg_begin = seg_begin;
+    g.ring = 1;
+    g.ring_step = t;
+    g.P = P;
+    g.fs = static_cast<int>(fs);
+    g.col_base = 0;
+    return g;
+}
+
+// One pass of the bf16 forward: K1 over the segments' hidden chunk, then K2
+// adding the chunk's partial output into the accumulator.
+template <int ACT>
+tsp_status_t fwd_pass_bf16(const void* X, const void* Wg, const void* Wu, const void* Wd,
+                           int64_t n, int64_t d, int64_t f, const SegGeom& g, int64_t width,
+                           int mode, __nv_bfloat16* H, float* acc, void* Y, cudaStream_t st,
+                           int dev, int sms) {
+    using K1 = FwdHidden<ACT>;
+    using K2 = DownAccum<true, 1>;
+    typename K1::Params p1;
+    std::memset(&p1, 0, sizeof(p1));
+    if (!tmap_bf16(&p1.tmX, X, d, n, d, 64, 128, SW128) ||
+        !tmap_bf16(&p1.tmG, Wg, f, d, f, 64, 64, SW128) ||
+        (ACT == 1 && !tmap_bf16(&p1.tmU, Wu, f, d, f, 64, 64, SW128)))
+        return TSP_ERR_CUDA;
+    p1.g = g;
+    p1.d = static_cast<int>(d);
+    p1.width = static_cast<int>(width);
+    p1.H = H;
+    p1.ldh = width;
+    TSP_TRY(launch_umma<K1>(p1, st, dev, sms));
+
+    typename K2::Params p2;
+    std::memset(&p2, 0, sizeof(p2));
+    const int64_t hrows = static_cast<int64_t>(g.num_segs) * g.seg_rows;
+    if (!tmap_bf16(&p2.tmA0, H, width, hrows, width, 64, 128, SW128) ||
+        !tmap_bf16(&p2.tmB0, Wd, d, f, d, 64, 64, SW128))
+        return TSP_ERR_CUDA;
+    p2.g = g;
+    p2.kdim = static_cast<int>(width);
+    p2.n_out = static_cast<int>(d);
+    p2.mode = mode;
+    p2.acc = acc;
+    p2.ldacc = d;
+    p2.out = static_cast<__nv_bfloat16*>(Y);
+    p2.ldo = d;
+    return launch_umma<K2>(p2, st, dev, sms);
+}
+
+template <int ACT>
+tsp_status_t forward_bf16(const void* X, const void* Wg, const void* Wu, const void* Wd, int64_t n,
+                          int64_t d, int64_t f, int P, const FwdPlan& pl, void* Y, void* ws,
+                          cudaStream_t st, int dev, int sms) {
+    auto* H = static_cast<__nv_bfloat16*>(ws);
+    float* acc = pl.acc_bytes ? reinterpret_cast<float*>(static_cast<char*>(ws) +
+                                                         align256(pl.h_bytes))
+                              : nullptr;
+    const int64_t fs = f / P;
+    if (!pl.ring) {
+        const int np = static_cast<int>(pl.chunks.size());
+        for (int i = 0; i < np; ++i) {
+            const SegGeom g = seg_all_rows(n, P, fs, pl.chunks[i].col_base);
+            TSP_TRY(fwd_pass_bf16<ACT>(X, Wg, Wu, Wd, n, d, f, g, pl.chunks[i].width,
+                                       accum_mode(i, np), H, acc, Y, st, dev, sms));
+        }
+    } else {
+        for (int t = 0; t < P; ++t)
+            for (int s0 = 0; s0 < P; s0 += pl.tsp_group) {
+                const int cnt = std::min(pl.tsp_group, P - s0);
+                const SegGeom g = seg_ring(n, P, fs, s0, cnt, t);
+                TSP_TRY(fwd_pass_bf16<ACT>(X, Wg, Wu, Wd, n, d, f, g, fs, accum_mode(t, P), H, acc,
+                                           Y, st, dev, sms));
+            }
+    }
+    return TSP_OK;
+}
+
+tsp_status_t forward_f32(const float* X, const float* Wg, const float* Wu, const float* Wd,
+                         int64_t n, int64_t d, int64_t f, int P, tsp_act_t act, const FwdPlan& pl,
+                         float* Y, void* ws, cudaStream_t st) {
+    float* H = static_cast<float*>(ws);
+    const int64_t fs = f / P;
+    auto run = [&](const SegGeom& g, int64_t width, int first) -> tsp_status_t {
+        dim3 gh(static_cast<unsigned>((width + kF32Tile - 1) / kF32Tile),
+                static_cast<unsigned>((g.seg_rows + kF32Tile - 1) / kF32Tile),
+                static_cast<unsigned>(g.num_segs));
+        TraceRec rec;
+        bool traced = trace_begin(st, &rec, act == TSP_ACT_SWIGLU ? "f32_hidden_swiglu" : "f32_hidden_gelu");
+        if (act == TSP_ACT_SWIGLU)
+            f32_hidden_kernel<1><<<gh, 256, 0, st>>>(X, Wg, Wu, static_cast<int>(d),
+                                                     static_cast<int>(f), g, static_cast<int>(width),
+                                                     H, width);
+        else
+            f32_hidden_kernel<0><<<gh, 256, 0, st>>>(X, Wg, Wu, static_cast<int>(d),
+                                                     static_cast<int>(f), g, static_cast<int>(width),
+                                                     H, width);
+        if (traced) trace_end(st, &rec);
+        if (cudaGetLastError() != cudaSuccess) return TSP_ERR_CUDA;
+        dim3 gd(static_cast<unsigned>((d + kF32Tile - 1) / kF32Tile),
+                static_cast<unsigned>((g.seg_rows + kF32Tile - 1) / kF32Tile),
+                static_cast<unsigned>(g.num_segs));
+        traced = trace_begin(st, &rec, "f32_down");
+        f32_down_kernel<<<gd, 256, 0, st>>>(H, width, Wd, static_cast<int>(d), g,
+                                            static_cast<int>(width), first, Y);
+        if (traced) trace_end(st, &rec);
+        return cudaGetLastError() == cudaSuccess ? TSP_OK : TSP_ERR_CUDA;
+    };
+    if (!pl.ring) {
+        for (size_t i = 0; i < pl.chunks.size(); ++i)
+            TSP_TRY(run(seg_all_rows(n, P, fs, pl.chunks[i].col_base), pl.chunks[i].width, i == 0));
+    } else {
+        for (int t = 0; t < P; ++t) TSP_TRY(run(seg_ring(n, P, fs, 0, P, t), fs, t == 0));
+    }
+    return TSP_OK;
+}
+
+// ---------------------------------------------------------------------------
+// backward (bf16, weight-shard schedule)
+
+struct BwdPlan {
+    bool ok = true;
+    std::vector<Chunk> chunks;
+    size_t buf_bytes = 0;  // one of H / dG / dU
+    int nbufs = 3;
+    size_t acc_bytes = 0;
+    size_t total() const { return nbufs * align256(buf_bytes) + align256(acc_bytes); }
+};
+
+BwdPlan plan_backward_budget(int64_t n, int64_t d, int64_t f, int P, tsp_act_t act, size_t budget) {
+    BwdPlan pl;
+    pl.nbufs = act == TSP_ACT_SWIGLU ? 3 : 2;
+    const int64_t mc = max_chunk_cols(budget, static_cast<size_t>(n) * 2 * pl.nbufs);
+    if (mc == 0) {
+        pl.ok = false;
+        return pl;
+    }
+    pl.chunks = plan_chunks(f, P, mc);
+    int64_t wmax = 0;
+    for (auto& c : pl.chunks) wmax = std::max(wmax, c.width);
+    pl.buf_bytes = static_cast<size_t>(n) * wmax * 2;
+    pl.acc_bytes = pl.chunks.size() > 1 ? static_cast<size_t>(n) * d * 4 : 0;
+    return pl;
+}
+
+BwdPlan plan_backward(int64_t n, int64_t d, int64_t f, int P, tsp_act_t act) {
+    return plan_backward_budget(n, d, f, P, act, kBwdHiddenBudget);
+}
+
+BwdPlan plan_backward_for(int64_t n, int64_t d, int64_t f, int P, tsp_act_t act, size_t ws_bytes) {
+    BwdPlan pl = plan_backward(n, d, f, P, act);
+    if (pl.total() <= ws_bytes) return pl;
+    const size_t acc = align256(static_cast<size_t>(n) * d * 4);
+    if (ws_bytes <= acc + 1024) {
+        pl.ok = false;
+        return pl;
+    }
+    pl = plan_backward_budget(n, d, f, P, act, ws_bytes - acc - 1024);
+    if (pl.total() > ws_bytes) pl.ok = false;
+    return pl;
+}
+
+template <int ACT>
+tsp_status_t backward_bf16(const void* X, const void* Wg, const void* Wu, const void* Wd,
+                           const void* dY, int64_t n, int64_t d, int64_t f, int P,
+                           const BwdPlan& pl, void* dX, float* dWg, float* dWu, float* dWd,
+                           void* ws, cudaStream_t st, int dev, int sms) {
+    char* w = static_cast<char*>(ws);
+    const size_t bb = align256(pl.buf_bytes);
+    auto* Hc = reinterpret_cast<__nv_bfloat16*>(w);
+    auto* dGc = reinterpret_cast<__nv_bfloat16*>(w + bb);
+    auto* dUc = ACT == 1 ? reinterpret_cast<__nv_bfloat16*>(w + 2 * bb) : nullptr;
+    float* acc = pl.acc_bytes ? reinterpret_cast<float*>(w + pl.nbufs * bb) : nullptr;
+    const int64_t fs = f / P;
+    const int np = static_cast<int>(pl.chunks.size());
+    for (int i = 0; i < np; ++i) {
+        const int64_t cb = pl.chunks[i].col_base, C = pl.chunks[i].width;
+        // K3: recompute G (U), dH; emit H, dG (dU)
+        {
+            using K = BwdHidden<ACT>;
+            typename K::Params p;
+            std::memset(&p, 0, sizeof(p));
+            if (!tmap_bf16(&p.tmX, X, d, n, d, 32, 128, SW64) ||
+                !tmap_bf16(&p.tmDY, dY, d, n, d, 32, 128, SW64) ||
+                !tmap_bf16(&p.tmG, Wg, f, d, f, 64, 32, SW128) ||
+                (ACT == 1 && !tmap_bf16(&p.tmU, Wu, f, d, f, 64, 32, SW128)) ||
+                !tmap_bf16(&p.tmD, Wd, d, f, d, 32, 128, SW64))
+                return TSP_ERR_CUDA;
+            p.n = static_cast<int>(n);
+            p.d = static_cast<int>(d);
+            p.col_base = static_cast<int>(cb);
+            p.width = static_cast<int>(C);
+            p.H = Hc;
+            p.dG = dGc;
+            p.dU = dUc;
+            p.ld = C;
+            TSP_TRY(launch_umma<K>(p, st, dev, sms));
+        }
+        // K4a: dW_down[cb .. cb+C) = H^T . dY
+        {
+            using K = Wgrad<256, false>;
+            typename K::Params p;
+            std::memset(&p, 0, sizeof(p));
+            if (!tmap_bf16(&p.tmA, Hc, C, n, C, 64, 64, SW128) ||
+                !tmap_bf16(&p.tmB0, dY, d, n, d, 64, 64, SW128))
+                return TSP_ERR_CUDA;
+            p.ntok = static_cast<int>(n);
+            p.m_valid = static_cast<int>(C);
+            p.n_valid = static_cast<int>(d);
+            p.out0 = dWd;
+            p.ldo = d;
+            p.out_row0 = static_cast<int>(cb);
+            p.out_col0 = 0;
+            TSP_TRY(launch_umma<K>(p, st, dev, sms));
+        }
+        // K4b: dW_gate (dW_up)[:, cb .. cb+C) = X^T . dG (dU)
+        if (ACT == 1) {
+            using K = Wgrad<256, true>;
+            typename K::Params p;
+            std::memset(&p, 0, sizeof(p));
+            if (!tmap_bf16(&p.tmA, X, d, n, d, 64, 64, SW128) ||
+                !tmap_bf16(&p.tmB0, dGc, C, n, C, 64, 64, SW128) ||
+                !tmap_bf16(&p.tmB1, dUc, C, n, C, 64, 64, SW128))
+                return TSP_ERR_CUDA;
+            p.ntok = static_cast<int>(n);
+            p.m_valid = static_cast<int>(d);
+            p.n_valid = static_cast<int>(C);
+            p.out0 = dWg;
+            p.out1 = dWu;
+            p.ldo = f;
+            p.out_row0 = 0;
+            p.out_col0 = static_cast<int>(cb);
+            TSP_TRY(launch_umma<K>(p, st, dev, sms));
+        } else {
+            using K = Wgrad<128, false>;
+            typename K::Params p;
+            std::memset(&p, 0, sizeof(p));
+            if (!tmap_bf16(&p.tmA, X, d, n, d, 64, 64, SW128) ||
+                !tmap_bf16(&p.tmB0, dGc, C, n, C, 64, 64, SW128))
+                return TSP_ERR_CUDA;
+            p.ntok = static_cast<int>(n);
+            p.m_valid = static_cast<int>(d);
+            p.n_valid = static_cast<int>(C);
+            p.out0 = dWg;
+            p.ldo = f;
+            p.out_row0 = 0;
+            p.out_col0 = static_cast<int>(cb);
+            TSP_TRY(launch_umma<K>(p, st, dev, sms));
+        }
+        // K5: dX (+)= dG . W_gate[:, chunk]^T (+ dU . W_up[:, chunk]^T)
+        {
+            using K = DownAccum<false, ACT == 1 ? 2 : 1>;
+            typename K::Params p;
+            std::memset(&p, 0, sizeof(p));
+            if (!tmap_bf16(&p.tmA0, dGc, C, n, C, 64, 128, SW128) ||
+                !tmap_bf16(&p.tmB0, Wg, f, d, f, 64, 256, SW128))
+                return TSP_ERR_CUDA;
+            if (ACT == 1 && (!tmap_bf16(&p.tmA1, dUc, C, n, C, 64, 128, SW128) ||
+                             !tmap_bf16(&p.tmB1, Wu, f, d, f, 64, 256, SW128)))
+                return TSP_ERR_CUDA;
+            p.g = seg_all_rows(n, P, fs, cb);
+            p.kdim = static_cast<int>(C);
+            p.n_out = static_cast<int>(d);
+            p.mode = accum_mode(i, np);
+            p.acc = acc;
+            p.ldacc = d;
+            p.out = static_cast<__nv_bfloat16*>(dX);
+            p.ldo = d;
+            TSP_TRY(launch_umma<K>(p, st, dev, sms));
+        }
+    }
+    return TSP_OK;
+}
+
+}  // namespace
+}  // namespace tspmlp
+
+using namespace tspmlp;
+
+extern "C" {
+
+const char* tsp_status_string(tsp_status_t s) {
+    switch (s) {
+        case TSP_OK: return "ok";
+        case TSP_ERR_INVALID_ARG: return "invalid argument";
+        case TSP_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+        case TSP_ERR_ARCH: return "device is not compute capability 10.0 (B200, sm_100a)";
+        case TSP_ERR_CUDA: return "CUDA error";
+        case TSP_ERR_TIMEOUT: return "a device-side wait timed out";
+        case TSP_ERR_WORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+tsp_status_t tsp_mlp_workspace_size(int64_t n, int64_t d, int64_t f, int P, tsp_act_t act,
+                                    tsp_dtype_t dt, tsp_sched_t sched, int backward,
+                                    size_t* bytes) {
+    if (!bytes) return TSP_ERR_INVALID_ARG;
+    TSP_TRY(validate_shape(n, d, f, P, act, dt, sched));
+    if (backward) {
+        if (dt != TSP_DT_BF16 || sched != TSP_SCHED_WEIGHT_SHARDS) return TSP_ERR_INVALID_ARG;
+        *bytes = plan_backward(n, d, f, P, act).total();
+    } else {
+        *bytes = plan_forward(n, d, f, P, dt, sched).total();
+    }
+    return TSP_OK;
+}
+
+tsp_status_t tsp_mlp_forward_ex(const void* X, const void* Wg, const void* Wu, const void* Wd,
+                                int64_t n, int64_t d, int64_t f, int P, tsp_act_t act,
+                                tsp_dtype_t dt, tsp_sched_t sched, void* Y, void* ws,
+                                size_t ws_bytes, tsp_stream_t stream) {
+    TSP_TRY(validate_forward(X, Wg, Wu, Wd, n, d, f, P, act, dt, sched, Y));
+    const FwdPlan pl = plan_forward_for(n, d, f, P, dt, sched, ws ? ws_bytes : 0);
+    const size_t need = pl.total();
+    if (!pl.ok) return TSP_ERR_WORKSPACE;
+    if (need > 0) {
+        if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) return TSP_ERR_WORKSPACE;
+        const size_t e = dt == TSP_DT_BF16 ? 2 : 4;
+        const size_t xb = n * d * e, wb = d * f * e;
+        if (overlaps(ws, need, X, xb) || overlaps(ws, need, Wg, wb) || overlaps(ws, need, Wu, wb) ||
+            overlaps(ws, need, Wd, wb) || overlaps(ws, need, Y, xb))
+            return TSP_ERR_INVALID_ARG;
+    }
+    int dev = 0;
+    DevInfo di;
+    TSP_TRY(current_device(&dev, &di));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (dt == TSP_DT_F32)
+        return forward_f32(static_cast<const float*>(X), static_cast<const float*>(Wg),
+                           static_cast<const float*>(Wu), static_cast<const float*>(Wd), n, d, f, P,
+                           act, pl, static_cast<float*>(Y), ws, st);
+    if (act == TSP_ACT_SWIGLU)
+        return forward_bf16<1>(X, Wg, Wu, Wd, n, d, f, P, pl, Y, ws, st, dev, di.sms);
+    return forward_bf16<0>(X, Wg, Wu, Wd, n, d, f, P, pl, Y, ws, st, dev, di.sms);
+}
+
+tsp_status_t tsp_mlp_forward(const void* X, const void* Wg, const void* Wu, const void* Wd,
+                             int64_t n, int64_t d, int64_t f, int P, tsp_act_t act, void* Y,
+                             tsp_stream_t stream) {
+    TSP_TRY(validate_forward(X, Wg, Wu, Wd, n, d, f, P, act, TSP_DT_BF16,
+                             TSP_SCHED_WEIGHT_SHARDS, Y));
+    const size_t need = plan_forward(n, d, f, P, TSP_DT_BF16, TSP_SCHED_WEIGHT_SHARDS).total();
+    int dev = 0;
+    DevInfo di;
+    TSP_TRY(current_device(&dev, &di));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    void* ws = nullptr;
+    if (need && cudaMallocAsync(&ws, need, st) != cudaSuccess) return TSP_ERR_CUDA;
+    const tsp_status_t s = tsp_mlp_forward_ex(X, Wg, Wu, Wd, n, d, f, P, act, TSP_DT_BF16,
+                                              TSP_SCHED_WEIGHT_SHARDS, Y, ws, need, stream);
+    if (ws && cudaFreeAsync(ws, st) != cudaSuccess && s == TSP_OK) return TSP_ERR_CUDA;
+    return s;
+}
+
+tsp_status_t tsp_mlp_backward_ex(const void* X, const void* Wg, const void* Wu, const void* Wd,
+                                 const void* dY, int64_t n, int64_t d, int64_t f, int P,
+                                 tsp_act_t act, void* dX, float* dWg, float* dWu, float* dWd,
+                                 void* ws, size_t ws_bytes, tsp_stream_t stream) {
+    TSP_TRY(validate_backward(X, Wg, Wu, Wd, dY, n, d, f, P, act, dX, dWg, dWu, dWd));
+    const BwdPlan pl = plan_backward_for(n, d, f, P, act, ws ? ws_bytes : 0);
+    const size_t need = pl.total();
+    if (!pl.ok || !ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u))
+        return TSP_ERR_WORKSPACE;
+    const size_t xb = n * d * 2, wb = d * f * 2, gw = d * f * 4;
+    const void* bufs[9] = {X, Wg, Wu, Wd, dY, dX, dWg, dWu, dWd};
+    const size_t sz[9] = {xb, wb, wb, wb, xb, xb, gw, gw, gw};
+    for (int i = 0; i < 9; ++i)
+        if (overlaps(ws, need, bufs[i], sz[i])) return TSP_ERR_INVALID_ARG;
+    int dev = 0;
+    DevInfo di;
+    TSP_TRY(current_device(&dev, &di));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (act == TSP_ACT_SWIGLU)
+        return backward_bf16<1>(X, Wg, Wu, Wd, dY, n, d, f, P, pl, dX, dWg, dWu, dWd, ws, st, dev,
+                                di.sms);
+    return backward_bf16<0>(X, Wg, Wu, Wd, dY, n, d, f, P, pl, dX, dWg, dWu, dWd, ws, st, dev,
+                            di.sms);
+}
+
+tsp_status_t tsp_mlp_backward(const void* X, const void* Wg, const void* Wu, const void* Wd,
+                              const void* dY, int64_t n, int64_t d, int64_t f, int P,
+                              tsp_act_t act, void* dX, float* dWg, float* dWu, float* dWd,
+                              tsp_stream_t stream) {
+    TSP_TRY(validate_backward(X, Wg, Wu, Wd, dY, n, d, f, P, act, dX, dWg, dWu, dWd));
+    const size_t need = plan_backward(n, d, f, P, act).total();
+    int dev = 0;
+    DevInfo di;
+    TSP_TRY(current_device(&dev, &di));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    void* ws = nullptr;
+    if (cudaMallocAsync(&ws, need, st) != cudaSuccess) return TSP_ERR_CUDA;
+    const tsp_status_t s = tsp_mlp_backward_ex(X, Wg, Wu, Wd, dY, n, d, f, P, act, dX, dWg, dWu,
+                                               dWd, ws, need, stream);
+    if (cudaFreeAsync(ws, st) != cudaSuccess && s == TSP_OK) return TSP_ERR_CUDA;
+    return s;
+}
+
+tsp_status_t tsp_trace_enable(int enable) {
+    std::lock_guard<std::mutex> lk(g_trace_mu);
+    g_trace_on = enable != 0;
+    return TSP_OK;
+}
+
+tsp_status_t tsp_trace_collect(tsp_kernel_stat_t* stats, int capacity, int* count) {
+    if (!count || capacity < 0 || (capacity > 0 && !stats)) return TSP_ERR_INVALID_ARG;
+    std::vector<TraceRec> pend;
+    {
+        std::lock_guard<std::mutex> lk(g_trace_mu);
+        pend.swap(g_trace_pending);
+    }
+    tsp_status_t st = TSP_OK;
+    std::vector<TraceStat> add;
+    for (auto& r : pend) {
+        float ms = 0.f;
+        if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess)
+            st = TSP_ERR_CUDA;
+        cudaEventDestroy(r.a);
+        cudaEventDestroy(r.b);
+        add.push_back({r.name, 1, static_cast<double>(ms)});
+    }
+    std::lock_guard<std::mutex> lk(g_trace_mu);
+    for (auto& a : add) {
+        bool found = false;
+        for (auto& t : g_trace_stats)
+            if (std::strcmp(t.name, a.name) == 0) {
+                t.launches += 1;
+                t.ms += a.ms;
+                found = true;
+                break;
+            }
+        if (!found) g_trace_stats.push_back(a);
+    }
+    int k = 0;
+    for (auto& t : g_trace_stats) {
+        if (k < capacity) stats[k] = tsp_kernel_stat_t{t.name, t.launches, t.ms};
+        ++k;
+    }
+    *count = std::min(k, capacity);
+    return st;
+}
+
+tsp_status_t tsp_trace_reset(void) {
+    std::vector<TraceRec> pend;
+    {
+        std::lock_guard<std::mutex> lk(g_trace_mu);
+        pend.swap(g_trace_pending);
+        g_trace_stats.clear();
+    }
+    for (auto& r : pend) {
+        cudaEventSynchronize(r.b);
+        cudaEventDestroy(r.a);
+        cudaEventDestroy(r.b);
+    }
+    return TSP_OK;
+}
+
+tsp_status_t tsp_poll_device_error(tsp_stream_t stream) {
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return TSP_ERR_CUDA;
+    uint32_t word = 0;
+    if (cudaMemcpyFromSymbol(&word, tspmlp::g_device_error, sizeof(word)) != cudaSuccess)
+        return TSP_ERR_CUDA;
+    if (word) {
+        const uint32_t zero = 0;
+        if (cudaMemcpyToSymbol(tspmlp::g_device_error, &zero, sizeof(zero)) != cudaSuccess)
+            return TSP_ERR_CUDA;
+        return TSP_ERR_TIMEOUT;
+    }
+    return TSP_OK;
+}
+
+}  // extern "C"

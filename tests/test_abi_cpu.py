@@ -1,0 +1,124 @@
+"""The C-ABI library builds, loads and exports every symbol include/tspmlp.h
+declares; host-side logic (workspace sizing, argument validation, status
+strings) behaves as the header documents.  No GPU is needed: every call here
+returns before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sequence_transformer_mlp_b200 as T
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tspmlp.h")
+
+
+def declared_symbols():
+    with open(HEADER) as fh:
+        text = fh.read()
+    return re.findall(r"TSP_API\s+[\w\s\*]+?\b(tsp_\w+)\s*\(", text)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sequence_transformer_mlp_b200 import build
+    build.build()
+    return T.load()
+
+
+def test_header_declares_the_api():
+    syms = set(declared_symbols())
+    assert {"tsp_mlp_forward", "tsp_mlp_forward_ex", "tsp_mlp_backward", "tsp_mlp_backward_ex",
+            "tsp_mlp_workspace_size", "tsp_status_string", "tsp_poll_device_error"} <= syms
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_status_strings(lib):
+    for code, name in T.STATUS_NAMES.items():
+        s = T.tsp_status_string(code)
+        assert isinstance(s, str) and s
+    assert T.tsp_status_string(0) == "ok"
+    assert T.tsp_status_string(99) == "unknown status"
+
+
+def test_workspace_sizes_follow_the_schedule(lib):
+    # fp32 weight-shard schedule: one shard's hidden block, Y accumulates in place
+    assert T.tsp_mlp_workspace_size(64, 128, 512, 2, "gelu", "f32") == 64 * 256 * 4
+    # bf16, a single chunk: no fp32 accumulator is needed
+    assert T.tsp_mlp_workspace_size(256, 64, 512, 1, "swiglu", "bf16") == 256 * 512 * 2
+    # Llama-3-8B shape, P = 8: chunks of whole shards within the hidden budget
+    n, d, f, P = 4096, 4096, 14336, 8
+    ws = T.tsp_mlp_workspace_size(n, d, f, P, "swiglu", "bf16")
+    acc = n * d * 4
+    h = ws - acc
+    assert h % (n * 2) == 0 and (h // (n * 2)) % (f // P) == 0
+    assert h <= 64 << 20
+    # TSP ring: the hidden block of a group of sequence shards plus the accumulator
+    wsr = T.tsp_mlp_workspace_size(32768, d, f, P, "swiglu", "bf16", "tsp_ring")
+    assert wsr > acc * 8 and (wsr - 32768 * d * 4) % (4096 * (f // P) * 2) == 0
+    # backward: H, dG, dU chunk buffers and the fp32 dX accumulator
+    wsb = T.tsp_mlp_workspace_size(n, d, f, P, "swiglu", "bf16", backward=True)
+    assert wsb > acc
+
+
+@pytest.mark.parametrize("args,code", [
+    ((0, 64, 128, 1, "gelu", "bf16"), 1),          # n <= 0
+    ((64, 64, 130, 4, "gelu", "bf16"), 2),         # d_ff % P
+    ((64, 60, 128, 1, "gelu", "bf16"), 2),         # d_model % 8 for bf16
+    ((64, 64, 128 * 3, 3, "gelu", "bf16"), 0),     # fine: d_ff/P = 128
+    ((64, 64, 108, 3, "gelu", "bf16"), 2),         # (d_ff/P) % 8 for bf16 (36)
+    ((64, 60, 120, 3, "gelu", "f32"), 0),          # fp32 takes any sizes
+    ((64, 64, 128, 5000, "gelu", "f32"), 2),       # P too large
+])
+def test_workspace_size_validation(lib, args, code):
+    out = ctypes.c_size_t(0)
+    n, d, f, P, act, dt = args
+    s = lib.tsp_mlp_workspace_size(n, d, f, P, T.ACT[act], T.DTYPE[dt], 0, 0, ctypes.byref(out))
+    assert s == code
+
+
+def test_tsp_ring_needs_divisible_tokens(lib):
+    out = ctypes.c_size_t(0)
+    assert lib.tsp_mlp_workspace_size(100, 64, 128, 8, 1, 0, 1, 0, ctypes.byref(out)) == 2
+    assert lib.tsp_mlp_workspace_size(96, 64, 128, 8, 1, 0, 1, 0, ctypes.byref(out)) == 0
+
+
+def test_bad_pointers_are_rejected_before_any_device_call(lib):
+    A, B, X, Y, U = 0x100000, 0x200000, 0x300000, 0x400000, 0x500000
+    # gelu with an up weight, swiglu without one, missing output
+    assert T.tsp_mlp_forward(X, A, U, B, 64, 64, 128, 1, "gelu", Y, stream=0, check=False) == 1
+    assert T.tsp_mlp_forward(X, A, None, B, 64, 64, 128, 1, "swiglu", Y, stream=0,
+                             check=False) == 1
+    assert T.tsp_mlp_forward(X, A, None, B, 64, 64, 128, 1, "gelu", None, stream=0,
+                             check=False) == 1
+    # Y overlapping X
+    assert T.tsp_mlp_forward_ex(X, A, None, B, 64, 64, 128, 1, "gelu", "bf16", "weight_shards",
+                                X + 64, 0x900000, 1 << 20, stream=0, check=False) == 1
+    # misaligned bf16 operand
+    assert T.tsp_mlp_forward_ex(X + 2, A, None, B, 64, 64, 128, 1, "gelu", "bf16",
+                                "weight_shards", Y, 0x900000, 1 << 20, stream=0,
+                                check=False) == 2
+    # workspace too small / missing
+    assert T.tsp_mlp_forward_ex(X, A, None, B, 64, 64, 128, 1, "gelu", "bf16", "weight_shards", Y,
+                                0x900000, 16, stream=0, check=False) == 6
+    assert T.tsp_mlp_forward_ex(X, A, None, B, 64, 64, 128, 1, "gelu", "bf16", "weight_shards", Y,
+                                None, 0, stream=0, check=False) == 6
+    # backward: dW_up must be NULL for gelu and given for swiglu; outputs must not alias
+    dX, g1, g2, g3 = 0x600000, 0x700000, 0x800000, 0xA00000
+    assert T.tsp_mlp_backward(X, A, None, B, Y, 64, 64, 128, 1, "gelu", dX, g1, g2, g3, stream=0,
+                              check=False) == 1
+    assert T.tsp_mlp_backward(X, A, U, B, Y, 64, 64, 128, 1, "swiglu", dX, g1, None, g3,
+                              stream=0, check=False) == 1
+    assert T.tsp_mlp_backward_ex(X, A, U, B, Y, 64, 64, 128, 1, "swiglu", dX, g1, g1, g3,
+                                 0xB00000, 1 << 30, stream=0, check=False) == 1
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(ImportError):
+        T.load(str(tmp_path / "nope.so"))
