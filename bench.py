@@ -1,0 +1,381 @@
+"""Benchmark of the sharded gated MLP on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+A step is one forward pass of the SwiGLU MLP of the Llama-3-8B shape
+(n=4096 tokens, d_model=4096, d_ff=14336, P=8 logical weight shards, bf16
+with fp32 accumulation) through the C ABI: gate/up projection with the fused
+activation, then the row-split down projection accumulated in place, shard
+chunk after shard chunk.  Other workloads (--workload) are for ad-hoc
+measurements; the default is the one the headline metric is quoted on.
+
+Timing: W untimed warm-up steps, then K steps bracketed by a barrier and
+torch.cuda.synchronize() on both sides, timed with CUDA events on the
+launching stream; the max over ranks is reported.  The weights alone (352 MB)
+exceed the 126 MB L2, so no flush is needed between steps.  Under torchrun
+(N > 1) every rank runs an independent replica (the path has no
+cross-device step), so scaling is weak and value = N x per-step FLOPs / max
+time.
+
+--impl reference times the fp64 CPU oracle on a bounded sample of token rows
+of the same workload (rank 0 only; other ranks exit at once).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import WORKLOADS, LLAMA8B, make_inputs  # noqa: E402
+
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
+KERNEL_SOURCES = ["ptx.cuh", "pipeline.cuh", "recipes.cuh"]
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            j = json.load(fh)
+        return {"bf16_tflops": j["bf16_tflops"], "bf16_tflops_sustained": j["bf16_tflops_sustained"],
+                "hbm_gbs": j["hbm_gbs"], "source": "measured"}
+    return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0,
+            "source": "fallback"}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "sequence_transformer_mlp_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel: str, wl_name: str, launches_per_step: int):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None
+    when there is none for this workload or the kernel sources changed since."""
+    if not os.path.exists(PROFILE_TRAFFIC):
+        return None
+    with open(PROFILE_TRAFFIC) as fh:
+        j = json.load(fh)
+    ent = j.get(wl_name, {}).get(kernel)
+    if not ent or ent.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi sampled every 200 ms while running (SM clock and throttle reasons)."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        try:
+            self.gpu = "GPU-" + str(torch.cuda.get_device_properties(gpu_index).uuid)
+        except Exception:  # pragma: no cover
+            self.gpu = str(gpu_index)
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.out.close()
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as fh:
+            for line in fh:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
+        loaded = [s for s in sm if s > 0.5 * smax] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def reference_arm(args, wl, rank):
+    """fp64 CPU oracle on a bounded sample of token rows of the workload."""
+    if rank != 0:
+        return
+    import oracle
+    inp = make_inputs(wl)
+    A, B = inp["A"].double().numpy(), inp["B"].double().numpy()
+    Wu = inp["Wu"].double().numpy() if inp["Wu"] is not None else None
+    rows = max(1, min(wl.n, args.ref_rows))
+    X = inp["X"][:rows].double().numpy()
+    per_row = wl.flops_forward() / wl.n
+
+    def step():
+        oracle.mlp_sharded(X, A, Wu, B, wl.act, wl.P)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    tflops = rows * per_row / dt / 1e12
+    sample = f"{rows} token rows of {wl.name} per step (sharded oracle, fp64)"
+    line = {
+        "impl": "reference", "metric": "sharded gated-MLP forward TFLOP/s", "value": tflops,
+        "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded torch.randn)",
+        "tokens_per_s": rows / dt,
+        "config": {"workload": wl.name, "n_tokens": wl.n, "d_model": wl.d, "d_ff": wl.f,
+                   "P": wl.P, "sample_rows": rows},
+        "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline(wl, target_s=12.0):
+    """The oracle, as it stands, on a bounded sample of rows (rank 0, N = 1)."""
+    import oracle
+    inp = make_inputs(wl)
+    A, B = inp["A"].double().numpy(), inp["B"].double().numpy()
+    Wu = inp["Wu"].double().numpy() if inp["Wu"] is not None else None
+    per_row = wl.flops_forward() / wl.n
+    probe = 32
+    t0 = time.perf_counter()
+    oracle.mlp_sharded(inp["X"][:probe].double().numpy(), A, Wu, B, wl.act, wl.P)
+    rate = probe / (time.perf_counter() - t0)
+    rows = int(max(probe, min(wl.n, rate * target_s)))
+    X = inp["X"][:rows].double().numpy()
+    t0 = time.perf_counter()
+    oracle.mlp_sharded(X, A, Wu, B, wl.act, wl.P)
+    dt = time.perf_counter() - t0
+    return {"value": rows * per_row / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"first {rows} token rows of {wl.name} (sharded fp64 oracle, {dt:.1f} s); "
+                      f"tokens/s {rows / dt:.1f}"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=LLAMA8B.name, choices=sorted(WORKLOADS))
+    ap.add_argument("--ref-rows", type=int, default=256)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    wl = WORKLOADS[args.workload]
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        reference_arm(args, wl, rank)
+        return
+
+    import sequence_transformer_mlp_b200 as T
+
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    inp = make_inputs(wl)
+    dev = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
+    n, d, f, P = wl.n, wl.d, wl.f, wl.P
+    sched = wl.sched
+    stream = torch.cuda.current_stream()
+    Y = torch.empty(n, d, dtype=torch.bfloat16, device="cuda")
+    need = T.tsp_mlp_workspace_size(n, d, f, P, wl.act, "bf16", sched, backward=wl.backward)
+    ws = torch.empty(max(need, 1), dtype=torch.uint8, device="cuda")
+    if wl.backward:
+        dX = torch.empty(n, d, dtype=torch.bfloat16, device="cuda")
+        dWg = torch.empty(d, f, dtype=torch.float32, device="cuda")
+        dWu = torch.empty(d, f, dtype=torch.float32, device="cuda")
+        dWd = torch.empty(f, d, dtype=torch.float32, device="cuda")
+        ws_f = torch.empty(max(T.tsp_mlp_workspace_size(n, d, f, P, wl.act, "bf16", sched), 1),
+                           dtype=torch.uint8, device="cuda")
+
+    def step(x=dev["X"]):
+        T.tsp_mlp_forward_ex(x, dev["A"], dev["Wu"], dev["B"], n, d, f, P, wl.act, "bf16", sched,
+                             Y, ws_f if wl.backward else ws,
+                             ws_f.numel() if wl.backward else need, stream)
+        if wl.backward:
+            T.tsp_mlp_backward_ex(x, dev["A"], dev["Wu"], dev["B"], dev["dY"], n, d, f, P, wl.act,
+                                  dX, dWg, dWu, dWd, ws, need, stream)
+
+    flops = wl.flops_forward() + (wl.flops_backward() if wl.backward else 0)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    assert T.tsp_poll_device_error() == T.TSP_OK
+
+    T.tsp_trace_reset()
+    T.tsp_trace_enable(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    T.tsp_trace_enable(False)
+    ms = e0.elapsed_time(e1) / args.steps
+    kstats = T.tsp_trace_collect()
+    T.tsp_trace_reset()
+    status = T.tsp_poll_device_error()
+    if status != T.TSP_OK:
+        raise SystemExit(f"device error {T.STATUS_NAMES.get(status)} during the timed region")
+
+    # end to end through the public call with host buffers: pinned X in, Y out
+    Xh = inp["X"].pin_memory()
+    Yh = torch.empty(n, d, dtype=torch.bfloat16).pin_memory()
+    Xd = torch.empty_like(dev["X"])
+    for _ in range(2):
+        Xd.copy_(Xh, non_blocking=True)
+        step(Xd)
+        Yh.copy_(Y, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for _ in range(args.steps):
+        Xd.copy_(Xh, non_blocking=True)
+        step(Xd)
+        Yh.copy_(Y, non_blocking=True)
+    e3.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_e2e = e2.elapsed_time(e3) / args.steps
+
+    if dist is not None:
+        t = torch.tensor([ms, ms_e2e], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, ms_e2e = t.tolist()
+
+    if rank == 0:
+        pk = peaks()
+        tflops = world * flops / (ms * 1e-3) / 1e12
+        # dominant kernel: the one with the largest share of traced time
+        total_k = sum(v[1] for v in kstats.values())
+        dom, (dom_launches, dom_ms) = max(kstats.items(), key=lambda kv: kv[1][1])
+        launches_total = sum(v[0] for v in kstats.values())
+        dom_flops_per_launch = kernel_flops_per_step(dom, wl) / (dom_launches / args.steps)
+        achieved = dom_flops_per_launch / (dom_ms / dom_launches * 1e-3) / 1e12
+        traffic = traffic_for(dom, wl.name, dom_launches // args.steps)
+        line = {
+            "metric": "sharded gated-MLP forward TFLOP/s" if not wl.backward
+            else "sharded gated-MLP forward+backward TFLOP/s",
+            "value": tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded torch.randn, cast to bf16)",
+            "tokens_per_s": world * n / (ms * 1e-3),
+            "pct_of_bf16_peak": 100.0 * tflops / (world * pk["bf16_tflops"]),
+            "pct_of_bf16_peak_sustained": 100.0 * tflops / (world * pk["bf16_tflops_sustained"]),
+            "config": {"workload": wl.name, "n_tokens": n, "d_model": d, "d_ff": f, "P": P,
+                       "act": wl.act, "schedule": sched, "parallelism": f"replicas{world}",
+                       "l2": "inputs larger than L2 (weights 3 x d x f bf16), no flush"},
+            "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved,
+                         "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": achieved / pk["bf16_tflops"],
+                         "frac_of_sustained": achieved / pk["bf16_tflops_sustained"],
+                         "peak_source": pk["source"], "traffic": traffic,
+                         "flops_per_launch": dom_flops_per_launch,
+                         "share_of_kernel_time": dom_ms / total_k if total_k else None},
+            "kernels": {k: {"launches": v[0], "ms_per_launch": v[1] / v[0]}
+                        for k, v in kstats.items()},
+            "gpu_launches": launches_total,
+            "e2e": {"value": world * flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": Xh.numel() * Xh.element_size(),
+                    "d2h_bytes_per_step": Yh.numel() * Yh.element_size(),
+                    "ms_per_step": ms_e2e},
+            "clocks": clk.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(wl)
+        print(json.dumps(line), flush=True)
+
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def kernel_flops_per_step(kernel: str, wl) -> float:
+    """Algorithmic FLOPs one step spends in `kernel` (2 x rows x cols x K of each
+    product it computes).  Per step the forward hidden kernel covers all n x f
+    hidden units once and the down kernel all n x d outputs over K = d_ff,
+    whatever the number of launches (chunks, ring steps) they are split into.
+    The backward hidden kernel's recomputed G/U products are counted: they run
+    on the tensor cores like the rest."""
+    n, d, f = wl.n, wl.d, wl.f
+    return {
+        "fwd_hidden_swiglu": 2 * 2 * n * d * f,
+        "fwd_hidden_gelu": 2 * n * d * f,
+        "down_accum_fwd": 2 * n * d * f,
+        "bwd_hidden_swiglu": 2 * 3 * n * d * f,
+        "bwd_hidden_gelu": 2 * 2 * n * d * f,
+        "wgrad_down": 2 * n * d * f,
+        "wgrad_gate_up": 2 * 2 * n * d * f,
+        "wgrad_gelu_a": 2 * n * d * f,
+        "dgrad_accum_swiglu": 2 * 2 * n * d * f,
+        "dgrad_accum_gelu": 2 * n * d * f,
+    }[kernel]
+
+
+if __name__ == "__main__":
+    main()

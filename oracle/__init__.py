@@ -168,16 +168,17 @@ def mlp_tsp(X, A, Wu, B, act: str, P: int, reverse: bool = False) -> np.ndarray:
     return Y
 
 
-def mlp_backward(X, A, Wu, B, dY, act: str):
-    """Returns (dX, dA, dWu, dB); dWu is None for the plain GeLU MLP."""
+def mlp_backward(X, A, Wu, B, dY, act: str, outputs=("dX", "dA", "dWu", "dB")):
+    """Returns (dX, dA, dWu, dB); dWu is None for the plain GeLU MLP, and any
+    gradient not named in ``outputs`` is None (and not computed)."""
     X, A, Wu, B, dY = map(_f64, (X, A, Wu, B, dY))
     n, d, f = _dims(X, A, Wu, B, act)
     if dY.shape != (n, d):
         raise ValueError("dY must be [n,d]")
-    dX = np.empty((n, d), np.float64)
-    dA = np.empty((d, f), np.float64)
-    dWu = np.empty((d, f), np.float64) if act == "swiglu" else None
-    dB = np.empty((f, d), np.float64)
+    dX = np.empty((n, d), np.float64) if "dX" in outputs else None
+    dA = np.empty((d, f), np.float64) if "dA" in outputs else None
+    dWu = np.empty((d, f), np.float64) if act == "swiglu" and "dWu" in outputs else None
+    dB = np.empty((f, d), np.float64) if "dB" in outputs else None
     _check(_load().oracle_mlp_backward(_p(X), _p(A), _p(Wu), _p(B), _p(dY), n, d, f, ACT[act],
                                        _p(dX), _p(dA), _p(dWu), _p(dB)), "oracle_mlp_backward")
     return dX, dA, dWu, dB

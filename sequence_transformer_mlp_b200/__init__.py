@@ -193,26 +193,32 @@ def tsp_trace_reset() -> None:
 # --------------------------------------------------------------------------- torch conveniences
 
 
+def _nbytes(t) -> int:
+    return t.numel() * t.element_size()
+
+
 def mlp_forward(X, W_gate, W_up, W_down, P: int, act: str, sched: str = "weight_shards",
                 out=None, workspace=None, stream=None):
     """Y = act-MLP(X) through tsp_mlp_forward_ex; dtype follows X (bf16 or fp32).
-    Allocates Y and the workspace with torch unless given."""
+    Allocates Y and the preferred workspace with torch unless given; a given
+    workspace tensor is passed with its own size (the schedule adapts to it)."""
     import torch
     n, d = X.shape
     f = W_gate.shape[1]
     dt = "bf16" if X.dtype == torch.bfloat16 else "f32"
     Y = out if out is not None else torch.empty((n, d), dtype=X.dtype, device=X.device)
-    need = tsp_mlp_workspace_size(n, d, f, P, act, dt, sched)
-    ws = workspace
-    if ws is None and need:
-        ws = torch.empty(need, dtype=torch.uint8, device=X.device)
+    if workspace is None:
+        need = tsp_mlp_workspace_size(n, d, f, P, act, dt, sched)
+        ws = torch.empty(need, dtype=torch.uint8, device=X.device) if need else None
+    else:
+        ws, need = workspace, _nbytes(workspace)
     tsp_mlp_forward_ex(X, W_gate, W_up, W_down, n, d, f, P, act, dt, sched, Y, ws, need, stream)
     return Y
 
 
 def mlp_backward(X, W_gate, W_up, W_down, dY, P: int, act: str, workspace=None, stream=None):
     """(dX bf16, dW_gate fp32, dW_up fp32 or None, dW_down fp32) through
-    tsp_mlp_backward_ex."""
+    tsp_mlp_backward_ex; a given workspace tensor is passed with its own size."""
     import torch
     n, d = X.shape
     f = W_gate.shape[1]
@@ -221,8 +227,11 @@ def mlp_backward(X, W_gate, W_up, W_down, dY, P: int, act: str, workspace=None, 
     dWg = torch.empty((d, f), dtype=torch.float32, device=dev)
     dWu = torch.empty((d, f), dtype=torch.float32, device=dev) if act == "swiglu" else None
     dWd = torch.empty((f, d), dtype=torch.float32, device=dev)
-    need = tsp_mlp_workspace_size(n, d, f, P, act, "bf16", "weight_shards", backward=True)
-    ws = workspace if workspace is not None else torch.empty(need, dtype=torch.uint8, device=dev)
+    if workspace is None:
+        need = tsp_mlp_workspace_size(n, d, f, P, act, "bf16", "weight_shards", backward=True)
+        ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    else:
+        ws, need = workspace, _nbytes(workspace)
     tsp_mlp_backward_ex(X, W_gate, W_up, W_down, dY, n, d, f, P, act, dX, dWg, dWu, dWd, ws, need,
                         stream)
     return dX, dWg, dWu, dWd
