@@ -71,7 +71,8 @@ typedef enum {
     TSP_ERR_ARCH = 3,              /* current device is not compute capability 10.0 */
     TSP_ERR_CUDA = 4,              /* a CUDA runtime call or launch failed */
     TSP_ERR_TIMEOUT = 5,           /* a bounded device-side wait ran out */
-    TSP_ERR_WORKSPACE = 6          /* workspace NULL or smaller than tsp_mlp_workspace_size */
+    TSP_ERR_WORKSPACE = 6,         /* workspace NULL or smaller than tsp_mlp_workspace_size */
+    TSP_ERR_SCRATCH_LIMIT = 7      /* needs more scratch than tsp_mlp_forward_noalloc holds */
 } tsp_status_t;
 
 typedef enum {
@@ -121,6 +122,30 @@ TSP_API tsp_status_t tsp_mlp_forward_ex(const void* X, const void* W_gate, const
                                 int64_t d_ff, int P, tsp_act_t act, tsp_dtype_t dtype,
                                 tsp_sched_t sched, void* Y, void* workspace,
                                 size_t workspace_bytes, tsp_stream_t stream);
+
+/* Forward pass that allocates nothing (bf16, weight-shard schedule).  The
+ * pages have no counterpart: this entry point exists for callers that cannot
+ * call cudaMalloc or cudaMallocAsync -- code running inside a host engine or
+ * plugin whose device memory is planned up front and must not grow, and code
+ * for which an allocation is unacceptable because it may synchronise the
+ * device and stall other streams.
+ * The scratch it needs (hidden chunk and fp32 accumulator) lives in a static
+ * device array of TSP_NOALLOC_SCRATCH_BYTES inside the library; every GPU that
+ * loads the library holds that array until the process exits.  The schedule is
+ * planned to fit the array; problems that need more (the fp32 accumulator
+ * alone is n_tokens * d_model * 4 bytes once the hidden layer takes more than
+ * one chunk) return TSP_ERR_SCRATCH_LIMIT before anything is launched.
+ * Arguments, requirements and results are those of tsp_mlp_forward.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  All calls on a device share the one array and it keeps the last
+ * call's contents; calls whose executions overlap on the GPU (different
+ * streams, or other threads) race on it and must be serialised by the caller. */
+#define TSP_NOALLOC_SCRATCH_BYTES (32u << 20)
+TSP_API tsp_status_t tsp_mlp_forward_noalloc(const void* X, const void* W_gate, const void* W_up,
+                                             const void* W_down, int64_t n_tokens,
+                                             int64_t d_model, int64_t d_ff, int P, tsp_act_t act,
+                                             void* Y, tsp_stream_t stream);
 
 /* Backward pass, bf16, weight-shard schedule, for upstream gradient dY.
  *   dY        [n_tokens][d_model] bf16

@@ -29,7 +29,9 @@ STATUS_NAMES = {
     4: "TSP_ERR_CUDA",
     5: "TSP_ERR_TIMEOUT",
     6: "TSP_ERR_WORKSPACE",
+    7: "TSP_ERR_SCRATCH_LIMIT",
 }
+NOALLOC_SCRATCH_BYTES = 32 << 20
 ACT = {"gelu": 0, "swiglu": 1}
 DTYPE = {"bf16": 0, "f32": 1}
 SCHED = {"weight_shards": 0, "tsp_ring": 1}
@@ -63,6 +65,7 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.tsp_mlp_forward.argtypes = [vp, vp, vp, vp, i64, i64, i64, ci, ci, vp, vp]
     lib.tsp_mlp_forward_ex.argtypes = [vp, vp, vp, vp, i64, i64, i64, ci, ci, ci, ci, vp, vp, sz,
                                        vp]
+    lib.tsp_mlp_forward_noalloc.argtypes = [vp, vp, vp, vp, i64, i64, i64, ci, ci, vp, vp]
     lib.tsp_mlp_backward.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, ci, ci, vp, vp, vp, vp,
                                      vp]
     lib.tsp_mlp_backward_ex.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, ci, ci, vp, vp, vp,
@@ -75,7 +78,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.tsp_trace_enable.argtypes = [ci]
     lib.tsp_trace_collect.argtypes = [ctypes.POINTER(KernelStat), ci, ctypes.POINTER(ci)]
     lib.tsp_trace_reset.argtypes = []
-    for name in ("tsp_mlp_forward", "tsp_mlp_forward_ex", "tsp_mlp_backward",
+    for name in ("tsp_mlp_forward", "tsp_mlp_forward_ex", "tsp_mlp_forward_noalloc",
+                 "tsp_mlp_backward",
                  "tsp_mlp_backward_ex", "tsp_mlp_workspace_size", "tsp_poll_device_error",
                  "tsp_trace_enable", "tsp_trace_collect", "tsp_trace_reset"):
         getattr(lib, name).restype = ci
@@ -130,6 +134,18 @@ def tsp_mlp_forward_ex(X, W_gate, W_up, W_down, n_tokens, d_model, d_ff, P, act,
                                   workspace_bytes, _stream(stream))
     if check:
         _check(s, "tsp_mlp_forward_ex")
+    return s
+
+
+def tsp_mlp_forward_noalloc(X, W_gate, W_up, W_down, n_tokens, d_model, d_ff, P, act, Y,
+                            stream=None, check=True) -> int:
+    """The forward pass without any allocation: its scratch is a static device
+    array of NOALLOC_SCRATCH_BYTES inside the library (see include/tspmlp.h)."""
+    s = load().tsp_mlp_forward_noalloc(_addr(X), _addr(W_gate), _addr(W_up), _addr(W_down),
+                                       n_tokens, d_model, d_ff, P, _enum(ACT, act), _addr(Y),
+                                       _stream(stream))
+    if check:
+        _check(s, "tsp_mlp_forward_noalloc")
     return s
 
 

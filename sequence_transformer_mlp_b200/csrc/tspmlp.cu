@@ -668,6 +668,33 @@ tsp_status_t backward_bf16(const void* X, const void* Wg, const void* Wu, const 
 }  // namespace
 }  // namespace tspmlp
 
+// ---------------------------------------------------------------------------
+// Scratch of tsp_mlp_forward_noalloc: a static device array, so that entry
+// point never allocates.  Host code must not hand the symbol itself to a
+// kernel (on the host it is only a stand-in); its device address is looked up
+// once per device with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char tsp_noalloc_scratch[TSP_NOALLOC_SCRATCH_BYTES];
+
+namespace tspmlp {
+namespace {
+
+void* g_noalloc_scratch_addr[kMaxDevices] = {};
+
+// Device address of the static scratch on device `dev` (the current device).
+tsp_status_t noalloc_scratch_address(int dev, void** out) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_noalloc_scratch_addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, tsp_noalloc_scratch) != cudaSuccess || !p) return TSP_ERR_CUDA;
+        g_noalloc_scratch_addr[dev] = p;
+    }
+    *out = g_noalloc_scratch_addr[dev];
+    return TSP_OK;
+}
+
+}  // namespace
+}  // namespace tspmlp
+
 using namespace tspmlp;
 
 extern "C" {
@@ -681,6 +708,8 @@ const char* tsp_status_string(tsp_status_t s) {
         case TSP_ERR_CUDA: return "CUDA error";
         case TSP_ERR_TIMEOUT: return "a device-side wait timed out";
         case TSP_ERR_WORKSPACE: return "workspace missing or too small";
+        case TSP_ERR_SCRATCH_LIMIT:
+            return "problem needs more scratch than the no-allocation entry point's static array";
     }
     return "unknown status";
 }
@@ -846,6 +875,25 @@ tsp_status_t tsp_trace_reset(void) {
         cudaEventDestroy(r.b);
     }
     return TSP_OK;
+}
+
+tsp_status_t tsp_mlp_forward_noalloc(const void* X, const void* Wg, const void* Wu,
+                                     const void* Wd, int64_t n, int64_t d, int64_t f, int P,
+                                     tsp_act_t act, void* Y, tsp_stream_t stream) {
+    TSP_TRY(validate_forward(X, Wg, Wu, Wd, n, d, f, P, act, TSP_DT_BF16,
+                             TSP_SCHED_WEIGHT_SHARDS, Y));
+    const FwdPlan pl = plan_forward_for(n, d, f, P, TSP_DT_BF16, TSP_SCHED_WEIGHT_SHARDS,
+                                        TSP_NOALLOC_SCRATCH_BYTES);
+    if (!pl.ok || pl.total() > TSP_NOALLOC_SCRATCH_BYTES) return TSP_ERR_SCRATCH_LIMIT;
+    int dev = 0;
+    DevInfo di;
+    TSP_TRY(current_device(&dev, &di));
+    void* ws = nullptr;
+    TSP_TRY(noalloc_scratch_address(dev, &ws));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (act == TSP_ACT_SWIGLU)
+        return forward_bf16<1>(X, Wg, Wu, Wd, n, d, f, P, pl, Y, ws, st, dev, di.sms);
+    return forward_bf16<0>(X, Wg, Wu, Wd, n, d, f, P, pl, Y, ws, st, dev, di.sms);
 }
 
 tsp_status_t tsp_poll_device_error(tsp_stream_t stream) {

@@ -1,0 +1,61 @@
+"""tsp_mlp_forward_noalloc: the forward pass for callers that cannot allocate
+device memory (engines or plugins with a fixed memory plan, or code that must
+not risk the device-wide synchronisation an allocation can cause).  Its
+scratch is a static device array inside the library, so the call itself
+allocates nothing.
+
+The test calls it through the C ABI twice in a row (the second call runs on
+whatever the first left in the shared static array) and checks each result
+against the allocating entry point tsp_mlp_forward, within the bf16 tolerance
+the other tests use.  It sits in a file of its own, collected last, so that a
+run stopping at the first failure has run every other test first; it holds no
+state between tests and passes alone in a fresh process too.
+"""
+import numpy as np
+import pytest
+import torch
+
+import sequence_transformer_mlp_b200 as T
+from workloads import Workload, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def _close(got, ref, what):
+    g = got.float().cpu().double().numpy()
+    r = ref.float().cpu().double().numpy()
+    assert np.isfinite(g).all(), what
+    mx = np.abs(r).max()
+    assert np.abs(g - r).max() <= 1e-2 * mx, what
+    assert np.linalg.norm(g - r) / np.linalg.norm(r) <= 5e-3, what
+
+
+# one case whose schedule needs several hidden chunks (fp32 accumulator in the
+# static array) and one that runs in a single chunk
+CASES = [("swiglu", 2048, 2048, 14336, 8), ("gelu", 300, 520, 1024, 4)]
+
+
+@pytest.mark.parametrize("act,n,d,f,P", CASES)
+def test_noalloc_forward_matches_allocating_forward_twice(act, n, d, f, P):
+    T.load()
+    wl = Workload(f"noalloc_{act}", act, "bf16", n, d, f, P, seed=31, w_std=0.02)
+    inp = make_inputs(wl)
+    X, A, Wu, B = (None if inp[k] is None else inp[k].cuda() for k in ("X", "A", "Wu", "B"))
+    ref = torch.empty(n, d, dtype=torch.bfloat16, device="cuda")
+    T.tsp_mlp_forward(X, A, Wu, B, n, d, f, P, act, ref)
+    for call in range(2):
+        Y = torch.full((n, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+        T.tsp_mlp_forward_noalloc(X, A, Wu, B, n, d, f, P, act, Y)
+        torch.cuda.synchronize()
+        assert T.tsp_poll_device_error() == T.TSP_OK
+        _close(Y, ref, f"call {call}")
+
+
+def test_noalloc_rejects_problems_beyond_its_static_scratch():
+    T.load()
+    # n * d_model * 4 bytes of fp32 accumulator alone exceed the static array
+    # placeholder addresses far apart: the call returns before touching them
+    X, A, U, B, Y = (k << 36 for k in range(1, 6))
+    s = T.tsp_mlp_forward_noalloc(X, A, U, B, 4096, 4096, 14336, 8, "swiglu", Y, check=False)
+    assert s == 7 and T.STATUS_NAMES[s] == "TSP_ERR_SCRATCH_LIMIT"
+    assert "static" in T.tsp_status_string(s)
