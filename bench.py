@@ -196,6 +196,44 @@ def cpu_baseline(wl, target_s=12.0):
                       f"tokens/s {rows / dt:.1f}"}
 
 
+def max_over_ranks(values, dist, device):
+    """Element-wise maximum of `values` over all ranks (every rank gets it)."""
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def replica_throughput(world: int, flops_per_step: float, ms_max: float) -> float:
+    """Whole-job TFLOP/s of `world` independent replicas timed by the slowest."""
+    return world * flops_per_step / (ms_max * 1e-3) / 1e12
+
+
+def end_to_end(args, inp, dev, step, Y, stream, barrier):
+    """The same step through the public call with host buffers: every step
+    copies X in from pinned host memory and reads Y back, all inside the
+    timed region.  Returns (ms per step, host X, host Y)."""
+    n, d = inp["X"].shape
+    Xh = inp["X"].pin_memory()
+    Yh = torch.empty(n, d, dtype=torch.bfloat16).pin_memory()
+    Xd = torch.empty_like(dev["X"])
+    for _ in range(2):
+        Xd.copy_(Xh, non_blocking=True)
+        step(Xd)
+        Yh.copy_(Y, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for _ in range(args.steps):
+        Xd.copy_(Xh, non_blocking=True)
+        step(Xd)
+        Yh.copy_(Y, non_blocking=True)
+    e3.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    return e2.elapsed_time(e3) / args.steps, Xh, Yh
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -205,6 +243,8 @@ def main():
     ap.add_argument("--workload", default=LLAMA8B.name, choices=sorted(WORKLOADS))
     ap.add_argument("--ref-rows", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the host-buffer loop (used for short profiler runs)")
     args = ap.parse_args()
     wl = WORKLOADS[args.workload]
 
@@ -282,34 +322,18 @@ def main():
         raise SystemExit(f"device error {T.STATUS_NAMES.get(status)} during the timed region")
 
     # end to end through the public call with host buffers: pinned X in, Y out
-    Xh = inp["X"].pin_memory()
-    Yh = torch.empty(n, d, dtype=torch.bfloat16).pin_memory()
-    Xd = torch.empty_like(dev["X"])
-    for _ in range(2):
-        Xd.copy_(Xh, non_blocking=True)
-        step(Xd)
-        Yh.copy_(Y, non_blocking=True)
-    torch.cuda.synchronize()
-    barrier()
-    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e2.record(stream)
-    for _ in range(args.steps):
-        Xd.copy_(Xh, non_blocking=True)
-        step(Xd)
-        Yh.copy_(Y, non_blocking=True)
-    e3.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    ms_e2e = e2.elapsed_time(e3) / args.steps
+    if args.no_e2e:
+        ms_e2e = float("nan")
+        Xh = Yh = None
+    else:
+        ms_e2e, Xh, Yh = end_to_end(args, inp, dev, step, Y, stream, barrier)
 
     if dist is not None:
-        t = torch.tensor([ms, ms_e2e], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, ms_e2e = t.tolist()
+        ms, ms_e2e = max_over_ranks([ms, ms_e2e], dist, "cuda")
 
     if rank == 0:
         pk = peaks()
-        tflops = world * flops / (ms * 1e-3) / 1e12
+        tflops = replica_throughput(world, flops, ms)
         # dominant kernel: the one with the largest share of traced time
         total_k = sum(v[1] for v in kstats.values())
         dom, (dom_launches, dom_ms) = max(kstats.items(), key=lambda kv: kv[1][1])
@@ -340,10 +364,11 @@ def main():
             "kernels": {k: {"launches": v[0], "ms_per_launch": v[1] / v[0]}
                         for k, v in kstats.items()},
             "gpu_launches": launches_total,
-            "e2e": {"value": world * flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
-                    "h2d_bytes_per_step": Xh.numel() * Xh.element_size(),
-                    "d2h_bytes_per_step": Yh.numel() * Yh.element_size(),
-                    "ms_per_step": ms_e2e},
+            "e2e": None if Xh is None else {
+                "value": replica_throughput(world, flops, ms_e2e), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": Xh.numel() * Xh.element_size(),
+                "d2h_bytes_per_step": Yh.numel() * Yh.element_size(),
+                "ms_per_step": ms_e2e},
             "clocks": clk.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:

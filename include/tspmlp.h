@@ -201,6 +201,19 @@ TSP_API tsp_status_t tsp_trace_collect(tsp_kernel_stat_t* stats, int capacity, i
 /* Drops all totals and pending events. */
 TSP_API tsp_status_t tsp_trace_reset(void);
 
+/* Failure-detection self-test; nothing faults, traps or hangs.
+ *   mode 0: a one-thread kernel waits on an mbarrier that nothing arrives on,
+ *           through the bounded wait every kernel of the library uses.
+ *   mode 1: one tile of the gate/up kernel whose producer arms its first stage
+ *           but leaves out that stage's loads, so the tensor-core pipeline
+ *           itself must give up: every role leaves through the abort path,
+ *           loads in flight are waited for, tensor memory is freed.
+ * Either kernel returns after about two seconds; the call returns TSP_OK once
+ * it is launched, and the following tsp_poll_device_error() reports
+ * TSP_ERR_TIMEOUT (and clears it).  Mode 1 allocates and frees its small
+ * buffers with cudaMallocAsync / cudaFreeAsync on `stream`. */
+TSP_API tsp_status_t tsp_selftest_timeout(int mode, tsp_stream_t stream);
+
 /* Synchronises `stream`, then reads and clears the current device's error
  * word: TSP_OK, TSP_ERR_TIMEOUT if a kernel gave up waiting, TSP_ERR_CUDA if
  * the stream reported an error. */

@@ -21,6 +21,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libtspmlp.so")
 
 TSP_OK = 0
+TSP_ERR_TIMEOUT = 5
 STATUS_NAMES = {
     0: "TSP_OK",
     1: "TSP_ERR_INVALID_ARG",
@@ -75,13 +76,15 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.tsp_status_string.argtypes = [ci]
     lib.tsp_status_string.restype = ctypes.c_char_p
     lib.tsp_poll_device_error.argtypes = [vp]
+    lib.tsp_selftest_timeout.argtypes = [ci, vp]
     lib.tsp_trace_enable.argtypes = [ci]
     lib.tsp_trace_collect.argtypes = [ctypes.POINTER(KernelStat), ci, ctypes.POINTER(ci)]
     lib.tsp_trace_reset.argtypes = []
     for name in ("tsp_mlp_forward", "tsp_mlp_forward_ex", "tsp_mlp_forward_noalloc",
                  "tsp_mlp_backward",
                  "tsp_mlp_backward_ex", "tsp_mlp_workspace_size", "tsp_poll_device_error",
-                 "tsp_trace_enable", "tsp_trace_collect", "tsp_trace_reset"):
+                 "tsp_trace_enable", "tsp_trace_collect", "tsp_trace_reset",
+                 "tsp_selftest_timeout"):
         getattr(lib, name).restype = ci
     if path is None:
         _lib = lib
@@ -187,6 +190,12 @@ def tsp_status_string(status: int) -> str:
 
 def tsp_poll_device_error(stream=None) -> int:
     return int(load().tsp_poll_device_error(_stream(stream)))
+
+
+def tsp_selftest_timeout(mode: int, stream=None) -> None:
+    """Launch the failure-detection self-test (see include/tspmlp.h); the next
+    tsp_poll_device_error() is expected to return TSP_ERR_TIMEOUT."""
+    _check(load().tsp_selftest_timeout(int(mode), _stream(stream)), "tsp_selftest_timeout")
 
 
 def tsp_trace_enable(enable: bool = True) -> None:

@@ -63,6 +63,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Self-test kernel: one thread waits on an mbarrier that nothing arrives on,
+// through the same bounded wait the pipeline uses; it gives up after
+// kWaitLimitNs and records a timeout in the device error word.
+__global__ void bounded_wait_selftest_kernel();
+
 // Waits for the phase of `bar` with parity `parity` to complete.  Returns
 // false (and records a timeout in the device error word) if it has not after
 // kWaitLimitNs, or false at once if *abort becomes non-zero.
@@ -208,6 +213,17 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
     return r;
+}
+
+__global__ void bounded_wait_selftest_kernel() {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        abort_flag = 0;
+        fence_barrier_init();
+        mbar_wait(smem_u32(&bar), 0, &abort_flag);
+    }
 }
 
 }  // namespace tspmlp

@@ -896,6 +896,50 @@ tsp_status_t tsp_mlp_forward_noalloc(const void* X, const void* Wg, const void* 
     return forward_bf16<0>(X, Wg, Wu, Wd, n, d, f, P, pl, Y, ws, st, dev, di.sms);
 }
 
+tsp_status_t tsp_selftest_timeout(int mode, tsp_stream_t stream) {
+    if (mode != 0 && mode != 1) return TSP_ERR_INVALID_ARG;
+    int dev = 0;
+    DevInfo di;
+    TSP_TRY(current_device(&dev, &di));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (mode == 0) {
+        bounded_wait_selftest_kernel<<<1, 32, 0, st>>>();
+        return cudaGetLastError() == cudaSuccess ? TSP_OK : TSP_ERR_CUDA;
+    }
+    // mode 1: a 128 x 256 x 128 gate/up problem -> one tile, four k-blocks
+    using K = FwdHidden<1>;
+    constexpr int64_t n = 128, d = 256, f = 128;
+    const size_t xb = n * d * 2, wb = d * f * 2, hb = n * f * 2;
+    char* buf = nullptr;
+    if (cudaMallocAsync(reinterpret_cast<void**>(&buf), xb + 2 * wb + hb, st) != cudaSuccess)
+        return TSP_ERR_CUDA;
+    tsp_status_t rc = TSP_OK;
+    if (cudaMemsetAsync(buf, 0, xb + 2 * wb + hb, st) != cudaSuccess) rc = TSP_ERR_CUDA;
+    typename K::Params p;
+    std::memset(&p, 0, sizeof(p));
+    if (rc == TSP_OK && (!tmap_bf16(&p.tmX, buf, d, n, d, 64, 128, SW128) ||
+                         !tmap_bf16(&p.tmG, buf + xb, f, d, f, 64, 64, SW128) ||
+                         !tmap_bf16(&p.tmU, buf + xb + wb, f, d, f, 64, 64, SW128)))
+        rc = TSP_ERR_CUDA;
+    if (rc == TSP_OK) {
+        p.g = seg_all_rows(n, 1, f, 0);
+        p.d = static_cast<int>(d);
+        p.width = static_cast<int>(f);
+        p.H = reinterpret_cast<__nv_bfloat16*>(buf + xb + 2 * wb);
+        p.ldh = f;
+        constexpr int smem = pipeline_smem_bytes<K>();
+        if (cudaFuncSetAttribute(umma_pipeline_kernel<K, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            rc = TSP_ERR_CUDA;
+        if (rc == TSP_OK) {
+            umma_pipeline_kernel<K, true><<<1, kPipelineThreads, smem, st>>>(p);
+            if (cudaGetLastError() != cudaSuccess) rc = TSP_ERR_CUDA;
+        }
+    }
+    if (cudaFreeAsync(buf, st) != cudaSuccess && rc == TSP_OK) rc = TSP_ERR_CUDA;
+    return rc;
+}
+
 tsp_status_t tsp_poll_device_error(tsp_stream_t stream) {
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (cudaStreamSynchronize(st) != cudaSuccess) return TSP_ERR_CUDA;
