@@ -241,6 +241,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=LLAMA8B.name, choices=sorted(WORKLOADS))
+    ap.add_argument("--sched", default=None, choices=["weight_shards", "tsp_ring", "shard_passes"],
+                    help="override the workload's schedule")
     ap.add_argument("--ref-rows", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true",
@@ -273,7 +275,7 @@ def main():
     inp = make_inputs(wl)
     dev = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
     n, d, f, P = wl.n, wl.d, wl.f, wl.P
-    sched = wl.sched
+    sched = args.sched or wl.sched
     stream = torch.cuda.current_stream()
     Y = torch.empty(n, d, dtype=torch.bfloat16, device="cuda")
     need = T.tsp_mlp_workspace_size(n, d, f, P, wl.act, "bf16", sched, backward=wl.backward)
@@ -389,6 +391,8 @@ def kernel_flops_per_step(kernel: str, wl) -> float:
     on the tensor cores like the rest."""
     n, d, f = wl.n, wl.d, wl.f
     return {
+        "fused_fwd_swiglu": 2 * 3 * n * d * f,
+        "fused_fwd_gelu": 2 * 2 * n * d * f,
         "fwd_hidden_swiglu": 2 * 2 * n * d * f,
         "fwd_hidden_gelu": 2 * n * d * f,
         "down_accum_fwd": 2 * n * d * f,

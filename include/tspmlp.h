@@ -84,12 +84,27 @@ typedef enum { TSP_DT_BF16 = 0, TSP_DT_F32 = 1 } tsp_dtype_t;
 
 typedef enum {
     /* Weight-shard schedule: every token meets shard 0, 1, ..., P-1 in order
-     * and the partial outputs accumulate in that order. */
+     * and the partial outputs accumulate in that order (the library picks its
+     * fastest implementation; today TSP_SCHED_SHARD_PASSES for bf16). */
     TSP_SCHED_WEIGHT_SHARDS = 0,
     /* Folded tensor-and-sequence ring: tokens form P equal sequence shards;
-     * at ring step t sequence shard s meets weight shard (s + t) mod P.
+     * at ring step t sequence shard s meets weight shard (s + t) mod P and
+     * adds its partial output into the shard's fp32 accumulator in place.
      * Needs n % P == 0. */
-    TSP_SCHED_TSP_RING = 1
+    TSP_SCHED_TSP_RING = 1,
+    /* Weight-shard schedule as separate passes: per chunk of shards one
+     * gate/up launch and one down-projection launch whose partial output is
+     * added into an fp32 [n][d_model] accumulator in place. */
+    TSP_SCHED_SHARD_PASSES = 2,
+    /* Weight-shard schedule as one persistent launch (bf16): per block of 128
+     * tokens the hidden activations go to a ring of row-block slots and the
+     * down projection's fp32 tensor-memory accumulator takes the shards'
+     * partial outputs in shard order.  Needs no [n][d_model] accumulator. */
+    TSP_SCHED_FUSED = 3,
+    /* The TSP ring as one persistent launch (bf16): as TSP_SCHED_FUSED, each
+     * sequence shard's K loop over the hidden units starting at its own weight
+     * shard.  Needs n % P == 0 and (d_ff / P) % 64 == 0. */
+    TSP_SCHED_TSP_RING_FUSED = 4
 } tsp_sched_t;
 
 /* Forward pass, bf16, weight-shard schedule.
@@ -107,7 +122,8 @@ TSP_API tsp_status_t tsp_mlp_forward(const void* X, const void* W_gate, const vo
 
 /* Forward pass with every option and a caller workspace.
  *   dtype      TSP_DT_BF16 (tensor cores) or TSP_DT_F32 (fp32 FMA; any sizes)
- *   sched      TSP_SCHED_WEIGHT_SHARDS or TSP_SCHED_TSP_RING (needs n % P == 0)
+ *   sched      a tsp_sched_t (the ring schedules need n % P == 0; the fused
+ *              ones bf16; TSP_SCHED_TSP_RING_FUSED also (d_ff / P) % 64 == 0)
  *   workspace  256-byte aligned device buffer, not overlapping any argument.
  *              tsp_mlp_workspace_size() gives the preferred size.  For bf16 a
  *              smaller workspace is accepted: the schedule then uses narrower
@@ -123,18 +139,20 @@ TSP_API tsp_status_t tsp_mlp_forward_ex(const void* X, const void* W_gate, const
                                 tsp_sched_t sched, void* Y, void* workspace,
                                 size_t workspace_bytes, tsp_stream_t stream);
 
-/* Forward pass that allocates nothing (bf16, weight-shard schedule).  The
+/* Forward pass that allocates nothing (bf16, TSP_SCHED_FUSED).  The
  * pages have no counterpart: this entry point exists for callers that cannot
  * call cudaMalloc or cudaMallocAsync -- code running inside a host engine or
  * plugin whose device memory is planned up front and must not grow, and code
  * for which an allocation is unacceptable because it may synchronise the
  * device and stall other streams.
- * The scratch it needs (hidden chunk and fp32 accumulator) lives in a static
- * device array of TSP_NOALLOC_SCRATCH_BYTES inside the library; every GPU that
- * loads the library holds that array until the process exits.  The schedule is
- * planned to fit the array; problems that need more (the fp32 accumulator
- * alone is n_tokens * d_model * 4 bytes once the hidden layer takes more than
- * one chunk) return TSP_ERR_SCRATCH_LIMIT before anything is launched.
+ * The scratch it needs (the ring of hidden-activation slots, 128 x d_ff bf16
+ * each, and the per-row-block counters of the fused schedule) lives in a
+ * static device array of TSP_NOALLOC_SCRATCH_BYTES inside the library; every
+ * GPU that loads the library holds that array until the process exits.  The
+ * ring is sized to fit the array; problems whose narrowest ring (three slots,
+ * or one per block of 128 tokens when there are fewer) does not fit -- d_ff
+ * above about 43,000 -- return TSP_ERR_SCRATCH_LIMIT before anything is
+ * launched.
  * Arguments, requirements and results are those of tsp_mlp_forward.
  * The first call on a device looks up the array's device address (once per
  * device, with that device current); make that first call before any stream

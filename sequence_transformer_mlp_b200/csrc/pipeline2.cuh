@@ -1,0 +1,314 @@
+// pipeline2.cuh -- the tcgen05 pipeline on CTA pairs (cta_group::2).
+//
+// A cluster of two CTAs on two SMs computes one 256 x 256 tile with paired
+// UMMAs (M = 256, N = 256, K = 16): CTA r of the pair stages rows
+// [128 r, 128 r + 128) of A and columns [128 r, 128 r + 128) of B in its own
+// shared memory, the leader (r = 0) issues every MMA, and each CTA's tensor
+// memory receives its own 128 rows of the accumulator.  Per SM a stage is
+// 32 KB for the same 128 x 256 x 64 of work that takes 48 KB on one CTA, so
+// the operand traffic from L2 into each SM drops by a third.
+//
+// Synchronisation across the pair:
+//   full[s]   leader only: the leader's producer expects the bytes of both
+//             CTAs' loads; both CTAs' TMA loads complete on it.
+//   empty[s]  both CTAs: the leader's commit arrives on both (multicast).
+//   tfull[b]  both CTAs: the leader's commit arrives on both (multicast).
+//   tempty[b] leader: the 4 epilogue warps of each CTA arrive (8 in all).
+// Every wait is bounded as in pipeline.cuh; a CTA whose partner stops
+// signalling times out on its own.  Both CTAs meet at a cluster barrier
+// before freeing tensor memory and leaving, so no CTA leaves while the
+// leader's MMAs may still read its shared memory.  No load uses cluster
+// multicast; only the commit arrivals are multicast.
+//
+// A pair recipe R supplies, like a recipe of pipeline.cuh: Params, kStages,
+// kStageBytes (per CTA), num_tiles, tile, num_kb, prefetch, and
+//   void load(const Params&, const Tile&, int kb, uint32_t rank, uint32_t stage,
+//             uint32_t leader_full_bar)               (1 thread in each CTA)
+//   void mma(const Tile&, int kb, uint32_t stage, uint32_t acc)   (leader, 1 thread)
+//   void epilogue(const Params&, const Tile&, uint32_t rank, uint32_t acc, int q, int lane)
+#pragma once
+
+#include "pipeline.cuh"
+
+namespace tspmlp {
+
+template <class R>
+constexpr int pair_smem_bytes() {
+    return R::kStages * R::kStageBytes + 256 + 1024;
+}
+
+template <class R>
+__global__ void __launch_bounds__(kPipelineThreads, 1)
+    umma_pair_pipeline_kernel(const __grid_constant__ typename R::Params p) {
+    constexpr int S = R::kStages;
+    constexpr int NB = 2;
+    constexpr uint32_t kAccCols = 256;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t ring = (raw + 1023u) & ~1023u;
+    uint8_t* ring_ptr = smem_raw + (ring - raw);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(ring_ptr + S * R::kStageBytes);
+    const uint32_t bar0 = smem_u32(bars);
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
+    auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * S + b); };
+    auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * S + NB + b); };
+    const uint32_t drain_bar = bar0 + 8u * (2 * S + 2 * NB);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 2 * NB + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        for (int b = 0; b < NB; ++b) {
+            mbar_init(tfull_bar(b), 1);
+            mbar_init(tempty_bar(b), 8);
+        }
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(smem_u32(tmem_slot), 512);
+        tmem_relinquish_pair();
+    }
+    if (warp == 0 && lane == 0) R::prefetch(p);
+    tc_fence_before();
+    cluster_sync_all();  // barrier inits and the allocation visible to both CTAs
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int num_tiles = R::num_tiles(p);
+    const int pair = static_cast<int>(cluster_id_x());
+    const int npairs = static_cast<int>(num_clusters_x());
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producers (both CTAs)
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0, armed = 0, armed_par = 0;
+            for (int t = pair; t < num_tiles && !*abort_flag; t += npairs) {
+                const auto ti = R::tile(p, t);
+                const int nkb = R::num_kb(p, ti);
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) break;
+                    if (leader) mbar_arrive_expect_tx(full_bar(stage), 2u * R::kStageBytes);
+                    R::load(p, ti, kb, rank, ring + stage * R::kStageBytes,
+                            map_to_cta(full_bar(stage), 0));
+                    armed |= 1u << stage;
+                    armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+                    if (++stage == S) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            // the leader's full barriers count both CTAs' loads: waiting on them
+            // lets every load of the pair land before shared memory goes away
+            if (leader)
+                for (int s = 0; s < S; ++s)
+                    if (armed & (1u << s)) mbar_wait_drain(full_bar(s), (armed_par >> s) & 1u);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (leader)
+        if (lane == 0 && leader) {
+            int stage = 0, local = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int t = pair; t < num_tiles && ok; t += npairs, ++local) {
+                const auto ti = R::tile(p, t);
+                const int nkb = R::num_kb(p, ti);
+                const int buf = local & 1;
+                const uint32_t use = static_cast<uint32_t>(local >> 1);
+                if (!mbar_wait(tempty_bar(buf), (use & 1u) ^ 1u, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t acc = tmem_base + static_cast<uint32_t>(buf) * kAccCols;
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait(full_bar(stage), phase, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    R::mma(ti, kb, ring + stage * R::kStageBytes, acc);
+                    umma_commit_pair_mc(empty_bar(stage), 0x3);
+                    if (++stage == S) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                umma_commit_pair_mc(tfull_bar(buf), 0x3);
+            }
+            umma_commit_pair_mc(drain_bar, 0x1);
+            mbar_wait_drain(drain_bar, 0);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue (both CTAs)
+        const int q = warp & 3;
+        int local = 0;
+        for (int t = pair; t < num_tiles; t += npairs, ++local) {
+            const int buf = local & 1;
+            const uint32_t use = static_cast<uint32_t>(local >> 1);
+            int ok = 0;
+            if (lane == 0) ok = mbar_wait(tfull_bar(buf), use & 1u, abort_flag) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            tc_fence_after();
+            const auto ti = R::tile(p, t);
+            R::epilogue(p, ti, rank, tmem_base + static_cast<uint32_t>(buf) * kAccCols, q, lane);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if (leader)
+                    mbar_arrive(tempty_bar(buf));
+                else
+                    mbar_arrive_remote(map_to_cta(tempty_bar(buf), 0));
+            }
+        }
+    }
+
+    tc_fence_before();
+    cluster_sync_all();  // no CTA leaves while the pair's MMAs may read its shared memory
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, 512);
+    }
+}
+
+// ============================================================================
+// Paired gate/up projection with the fused activation (see FwdHidden).
+// Tile = 256 token rows (128 per CTA).  SwiGLU: CTA 0 stages the gate columns,
+// CTA 1 the up columns of the same 128 hidden units, so TMEM columns 0-127
+// hold the gate and 128-255 the up pre-activations of each CTA's rows.
+// GeLU: 256 hidden units a tile, 128 staged by each CTA.
+template <int ACT>
+struct FwdHiddenPair {
+    using Params = typename FwdHidden<ACT>::Params;
+    static constexpr const char* kName = ACT == 1 ? "fwd_hidden_swiglu" : "fwd_hidden_gelu";
+    static constexpr int kBK = 64;
+    static constexpr int kOut = ACT == 1 ? 128 : 256;
+    static constexpr int kABytes = 128 * kBK * 2;
+    static constexpr int kStageBytes = kABytes + 128 * kBK * 2;
+    static constexpr int kStages = 6;
+    static constexpr uint32_t kIdesc = make_idesc_bf16(256, 256, false, true);
+    struct Tile {
+        int s, mi, nj;
+    };
+    __host__ __device__ static int pair_mtiles(const SegGeom& g) { return (g.seg_rows + 255) >> 8; }
+    __host__ __device__ static int ntiles_n(const Params& p) { return (p.width + kOut - 1) / kOut; }
+    __host__ __device__ static int num_tiles(const Params& p) {
+        return p.g.num_segs * pair_mtiles(p.g) * ntiles_n(p);
+    }
+    __device__ static Tile tile(const Params& p, int t) {
+        const int mt = pair_mtiles(p.g), per_seg = mt * ntiles_n(p);
+        const int s = t / per_seg, r = t - s * per_seg;
+        return Tile{s, r % mt, r / mt};
+    }
+    __device__ static int num_kb(const Params& p, const Tile&) { return (p.d + kBK - 1) / kBK; }
+    __device__ static void prefetch(const Params& p) { FwdHidden<ACT>::prefetch(p); }
+    __device__ static void load(const Params& p, const Tile& ti, int kb, uint32_t rank, uint32_t st,
+                                uint32_t bar) {
+        const int k0 = kb * kBK;
+        tma_load_2d_pair(st, &p.tmX, bar, k0,
+                         (p.g.seg_begin + ti.s) * p.g.seg_rows + ti.mi * 256 + rank * 128);
+        const int c = p.g.shard_col(ti.s) + ti.nj * kOut;
+        if (ACT == 1) {
+            const CUtensorMap* w = rank == 0 ? &p.tmG : &p.tmU;
+            tma_load_2d_pair(st + kABytes, w, bar, c, k0);
+            tma_load_2d_pair(st + kABytes + 8192, w, bar, c + 64, k0);
+        } else {
+            const int cr = c + static_cast<int>(rank) * 128;
+            tma_load_2d_pair(st + kABytes, &p.tmG, bar, cr, k0);
+            tma_load_2d_pair(st + kABytes + 8192, &p.tmG, bar, cr + 64, k0);
+        }
+    }
+    __device__ static void mma(const Tile&, int kb, uint32_t st, uint32_t acc) {
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t a = make_smem_desc(st + 32 * kk, 16, 1024, kLayoutSW128);
+            const uint64_t b = make_smem_desc(st + kABytes + 2048 * kk, 8192, 1024, kLayoutSW128);
+            umma_bf16_pair(acc, a, b, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+        }
+    }
+    __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t rank, uint32_t acc,
+                                    int q, int lane) {
+        // the same per-row work as the single-CTA tile, on this CTA's 128 rows
+        typename FwdHidden<ACT>::Tile t1{ti.s, 2 * ti.mi + static_cast<int>(rank), ti.nj};
+        FwdHidden<ACT>::epilogue(p, t1, acc, q, lane);
+    }
+};
+
+// ============================================================================
+// Paired down projection / input gradient with in-place fp32 accumulation
+// (see DownAccum).  Tile = 256 rows x 256 output columns; CTA r stages output
+// columns [128 r, 128 r + 128) of the B tile.
+template <bool B_MN, int NSEG>
+struct DownAccumPair {
+    using Base = DownAccum<B_MN, NSEG>;
+    using Params = typename Base::Params;
+    static constexpr const char* kName = Base::kName;
+    static constexpr int kBK = 64;
+    static constexpr int kABytes = 128 * kBK * 2;
+    static constexpr int kStageBytes = kABytes + 128 * kBK * 2;
+    static constexpr int kStages = 6;
+    static constexpr uint32_t kIdesc = make_idesc_bf16(256, 256, false, B_MN);
+    struct Tile {
+        int s, mi, nj;
+    };
+    __host__ __device__ static int pair_mtiles(const SegGeom& g) { return (g.seg_rows + 255) >> 8; }
+    __host__ __device__ static int ntiles_n(const Params& p) { return (p.n_out + 255) / 256; }
+    __host__ __device__ static int num_tiles(const Params& p) {
+        return p.g.num_segs * pair_mtiles(p.g) * ntiles_n(p);
+    }
+    __device__ static Tile tile(const Params& p, int t) {
+        const int mt = pair_mtiles(p.g), per_seg = mt * ntiles_n(p);
+        const int s = t / per_seg, r = t - s * per_seg;
+        return Tile{s, r % mt, r / mt};
+    }
+    __device__ static int num_kb(const Params& p, const Tile&) {
+        return NSEG * ((p.kdim + kBK - 1) / kBK);
+    }
+    __device__ static void prefetch(const Params& p) { Base::prefetch(p); }
+    __device__ static void load(const Params& p, const Tile& ti, int kb, uint32_t rank, uint32_t st,
+                                uint32_t bar) {
+        const int nkb1 = (p.kdim + kBK - 1) / kBK;
+        const int seg = NSEG > 1 ? kb / nkb1 : 0;
+        const int k = (kb - seg * nkb1) * kBK;
+        const CUtensorMap* ta = seg ? &p.tmA1 : &p.tmA0;
+        const CUtensorMap* tb = seg ? &p.tmB1 : &p.tmB0;
+        tma_load_2d_pair(st, ta, bar, k, ti.s * p.g.seg_rows + ti.mi * 256 + rank * 128);
+        const int kbase = p.g.shard_col(ti.s);
+        const int n0 = ti.nj * 256 + static_cast<int>(rank) * 128;
+        if (B_MN) {
+            tma_load_2d_pair(st + kABytes, tb, bar, n0, kbase + k);
+            tma_load_2d_pair(st + kABytes + 8192, tb, bar, n0 + 64, kbase + k);
+        } else {
+            tma_load_2d_pair(st + kABytes, tb, bar, kbase + k, n0);
+        }
+    }
+    __device__ static void mma(const Tile&, int kb, uint32_t st, uint32_t acc) {
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t a = make_smem_desc(st + 32 * kk, 16, 1024, kLayoutSW128);
+            const uint64_t b = B_MN ? make_smem_desc(st + kABytes + 2048 * kk, 8192, 1024, kLayoutSW128)
+                                    : make_smem_desc(st + kABytes + 32 * kk, 16, 1024, kLayoutSW128);
+            umma_bf16_pair(acc, a, b, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+        }
+    }
+    __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t rank, uint32_t acc,
+                                    int q, int lane) {
+        typename Base::Tile t1{ti.s, 2 * ti.mi + static_cast<int>(rank), ti.nj};
+        Base::epilogue(p, t1, acc, q, lane);
+    }
+};
+
+}  // namespace tspmlp

@@ -109,13 +109,16 @@ struct FwdHidden {
     struct Tile {
         int s, mi, nj;
     };
+    __host__ __device__ static int ntiles_n(const Params& p) { return (p.width + kOut - 1) / kOut; }
     __host__ __device__ static int num_tiles(const Params& p) {
-        return p.g.num_segs * p.g.mtiles() * ((p.width + kOut - 1) / kOut);
+        return p.g.num_segs * p.g.mtiles() * ntiles_n(p);
     }
+    // segment-major, then output slab, then row tile (row tiles fastest): one
+    // sequence segment's rows and weight shard at a time stay in L2
     __device__ static Tile tile(const Params& p, int t) {
-        const int mt = p.g.mtiles(), tm = p.g.num_segs * mt;
-        const int m = t % tm;
-        return Tile{m / mt, m % mt, t / tm};
+        const int mt = p.g.mtiles(), per_seg = mt * ntiles_n(p);
+        const int s = t / per_seg, r = t - s * per_seg;
+        return Tile{s, r % mt, r / mt};
     }
     __device__ static int num_kb(const Params& p, const Tile&) { return (p.d + kBK - 1) / kBK; }
     __device__ static void prefetch(const Params& p) {
@@ -220,13 +223,16 @@ struct DownAccum {
     struct Tile {
         int s, mi, nj;
     };
+    __host__ __device__ static int ntiles_n(const Params& p) { return (p.n_out + 255) / 256; }
     __host__ __device__ static int num_tiles(const Params& p) {
-        return p.g.num_segs * p.g.mtiles() * ((p.n_out + 255) / 256);
+        return p.g.num_segs * p.g.mtiles() * ntiles_n(p);
     }
+    // segment-major, then output slab, then row tile (row tiles fastest): one
+    // sequence segment's rows and weight shard at a time stay in L2
     __device__ static Tile tile(const Params& p, int t) {
-        const int mt = p.g.mtiles(), tm = p.g.num_segs * mt;
-        const int m = t % tm;
-        return Tile{m / mt, m % mt, t / tm};
+        const int mt = p.g.mtiles(), per_seg = mt * ntiles_n(p);
+        const int s = t / per_seg, r = t - s * per_seg;
+        return Tile{s, r % mt, r / mt};
     }
     __device__ static int num_kb(const Params& p, const Tile&) {
         return NSEG * ((p.kdim + kBK - 1) / kBK);

@@ -19,6 +19,8 @@
 #include <vector>
 
 #include "../../include/tspmlp.h"
+#include "fused.cuh"
+#include "pipeline2.cuh"
 #include "recipes.cuh"
 #include "simt_f32.cuh"
 
@@ -30,6 +32,7 @@ constexpr int kMaxDevices = 64;
 // Scratch budgets: the hidden chunk(s) of one pass should stay resident in the
 // 126 MB L2 between the producing and the consuming kernel.
 constexpr size_t kFwdHiddenBudget = 64ull << 20;   // one bf16 [rows][C] buffer
+constexpr size_t kFusedRingBudget = 96ull << 20;   // the fused schedule's H ring
 constexpr size_t kBwdHiddenBudget = 96ull << 20;   // H, dG, dU together
 
 struct DevInfo {
@@ -170,6 +173,59 @@ tsp_status_t launch_umma(const typename R::Params& p, cudaStream_t st, int dev, 
     return e == cudaSuccess ? TSP_OK : TSP_ERR_CUDA;
 }
 
+// Paired launch: clusters of two CTAs (cta_group::2 tiles), as many pairs as
+// can be resident at once, each walking the tile list persistently.
+template <class R>
+tsp_status_t launch_pair(const typename R::Params& p, cudaStream_t st, int dev, int sms) {
+    const int tiles = R::num_tiles(p);
+    if (tiles <= 0) return TSP_OK;
+    constexpr int smem = pair_smem_bytes<R>();
+    static_assert(smem <= 232448, "stage ring exceeds 227 KB of shared memory");
+    static bool attr_set[kMaxDevices] = {};
+    static int max_pairs[kMaxDevices] = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!attr_set[dev]) {
+            if (cudaFuncSetAttribute(umma_pair_pipeline_kernel<R>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     smem) != cudaSuccess)
+                return TSP_ERR_CUDA;
+            cudaLaunchConfig_t q = {};
+            q.gridDim = dim3(static_cast<unsigned>(sms / 2 * 2));
+            q.blockDim = dim3(kPipelineThreads);
+            q.dynamicSmemBytes = smem;
+            q.attrs = attr;
+            q.numAttrs = 1;
+            int nc = 0;
+            if (cudaOccupancyMaxActiveClusters(&nc, umma_pair_pipeline_kernel<R>, &q) != cudaSuccess ||
+                nc <= 0) {
+                cudaGetLastError();
+                nc = sms / 2;
+            }
+            max_pairs[dev] = nc;
+            attr_set[dev] = true;
+        }
+    }
+    const int pairs = std::min(tiles, max_pairs[dev]);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+    cfg.blockDim = dim3(kPipelineThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    TraceRec rec;
+    const bool traced = trace_begin(st, &rec, R::kName);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, umma_pair_pipeline_kernel<R>, p);
+    if (traced) trace_end(st, &rec);
+    return e == cudaSuccess ? TSP_OK : TSP_ERR_CUDA;
+}
+
 #define TSP_TRY(expr)                          \
     do {                                       \
         const tsp_status_t _s = (expr);        \
@@ -241,11 +297,16 @@ tsp_status_t validate_shape(int64_t n, int64_t d, int64_t f, int P, tsp_act_t ac
                             tsp_dtype_t dt, tsp_sched_t sched) {
     if (act != TSP_ACT_GELU && act != TSP_ACT_SWIGLU) return TSP_ERR_INVALID_ARG;
     if (dt != TSP_DT_BF16 && dt != TSP_DT_F32) return TSP_ERR_INVALID_ARG;
-    if (sched != TSP_SCHED_WEIGHT_SHARDS && sched != TSP_SCHED_TSP_RING) return TSP_ERR_INVALID_ARG;
+    if (sched < TSP_SCHED_WEIGHT_SHARDS || sched > TSP_SCHED_TSP_RING_FUSED)
+        return TSP_ERR_INVALID_ARG;
     if (n <= 0 || d <= 0 || f <= 0 || P <= 0) return TSP_ERR_INVALID_ARG;
     if (n > kMaxDim || d > kMaxDim || f > kMaxDim || P > 4096) return TSP_ERR_UNSUPPORTED_SHAPE;
     if (f % P != 0) return TSP_ERR_UNSUPPORTED_SHAPE;
-    if (sched == TSP_SCHED_TSP_RING && n % P != 0) return TSP_ERR_UNSUPPORTED_SHAPE;
+    const bool ring = sched == TSP_SCHED_TSP_RING || sched == TSP_SCHED_TSP_RING_FUSED;
+    if (ring && n % P != 0) return TSP_ERR_UNSUPPORTED_SHAPE;
+    if ((sched == TSP_SCHED_FUSED || sched == TSP_SCHED_TSP_RING_FUSED) && dt != TSP_DT_BF16)
+        return TSP_ERR_UNSUPPORTED_SHAPE;
+    if (sched == TSP_SCHED_TSP_RING_FUSED && (f / P) % 64 != 0) return TSP_ERR_UNSUPPORTED_SHAPE;
     if (dt == TSP_DT_BF16 && (d % 8 != 0 || (f / P) % 8 != 0)) return TSP_ERR_UNSUPPORTED_SHAPE;
     return TSP_OK;
 }
@@ -311,11 +372,48 @@ tsp_status_t validate_backward(const void* X, const void* Wg, const void* Wu, co
 struct FwdPlan {
     bool ok = true;
     bool ring = false;
-    std::vector<Chunk> chunks;  // weight-shard schedule
-    int tsp_group = 1;          // ring schedule: sequence shards per launch
+    // fused single-launch schedule (bf16)
+    bool fused = false;
+    int segs = 1, seg_rows = 0, mts = 0, MB = 0, GM = 1, R = 1;
+    size_t ring_bytes = 0, sync_bytes = 0;
+    // per-chunk pass schedule
+    std::vector<Chunk> chunks;  // weight-shard passes
+    int tsp_group = 1;          // ring passes: sequence shards per launch
     size_t h_bytes = 0, acc_bytes = 0;
-    size_t total() const { return align256(h_bytes) + align256(acc_bytes); }
+    size_t total() const {
+        return fused ? align256(ring_bytes) + align256(sync_bytes)
+                     : align256(h_bytes) + align256(acc_bytes);
+    }
 };
+
+// The fused schedule: row blocks of 128 tokens per sequence segment, grouped
+// GM at a time; the H ring holds three groups (R = 3*GM row-block slots, or one
+// per row block when that is fewer).  Larger groups re-read the weights fewer
+// times (once per group); GM is the largest of kFusedGroupRows that keeps the
+// ring within the budget.
+constexpr int kFusedGroupRows = 8;
+
+bool plan_fused(int64_t n, int64_t d, int64_t f, int P, bool ring, size_t budget, FwdPlan* pl) {
+    (void)d;
+    pl->fused = true;
+    pl->ring = ring;
+    pl->segs = ring ? P : 1;
+    pl->seg_rows = static_cast<int>(ring ? n / P : n);
+    pl->mts = (pl->seg_rows + 127) / 128;
+    pl->MB = pl->segs * pl->mts;
+    const size_t slot = static_cast<size_t>(128) * f * 2;
+    int GM = std::min(pl->MB, kFusedGroupRows);
+    int R = std::min(pl->MB, 3 * GM);
+    while (GM > 1 && static_cast<size_t>(R) * slot > budget) {
+        --GM;
+        R = std::min(pl->MB, 3 * GM);
+    }
+    pl->GM = GM;
+    pl->R = R;
+    pl->ring_bytes = static_cast<size_t>(R) * slot;
+    pl->sync_bytes = static_cast<size_t>(1 + 2 * pl->MB) * 4;
+    return pl->ring_bytes <= budget;
+}
 
 // Schedule of the forward pass for a hidden-buffer budget.  ok == false when
 // not even the narrowest schedule fits.
@@ -324,6 +422,10 @@ FwdPlan plan_forward_budget(int64_t n, int64_t d, int64_t f, int P, tsp_dtype_t 
     FwdPlan pl;
     const size_t e = dt == TSP_DT_BF16 ? 2 : 4;
     const int64_t fs = f / P;
+    if (dt == TSP_DT_BF16 && (sched == TSP_SCHED_FUSED || sched == TSP_SCHED_TSP_RING_FUSED)) {
+        pl.ok = plan_fused(n, d, f, P, sched == TSP_SCHED_TSP_RING_FUSED, budget, &pl);
+        return pl;
+    }
     if (sched == TSP_SCHED_TSP_RING) {
         pl.ring = true;
         const size_t per_seg = static_cast<size_t>(n / P) * fs * e;
@@ -355,17 +457,30 @@ FwdPlan plan_forward_budget(int64_t n, int64_t d, int64_t f, int P, tsp_dtype_t 
     return pl;
 }
 
-// The preferred schedule: hidden buffers within the L2-sized budget.
+// The preferred schedule: hidden buffers within their budgets.
 FwdPlan plan_forward(int64_t n, int64_t d, int64_t f, int P, tsp_dtype_t dt, tsp_sched_t sched) {
+    FwdPlan pl = plan_forward_budget(n, d, f, P, dt, sched, kFusedRingBudget);
+    if (pl.fused) return pl;
     return plan_forward_budget(n, d, f, P, dt, sched, kFwdHiddenBudget);
 }
 
 // The schedule for a caller workspace of ws_bytes: the preferred one if it
-// fits, otherwise narrower hidden chunks (bf16 only).
+// fits, otherwise a narrower one (bf16 only): fewer H-ring slots for the fused
+// schedule, narrower hidden chunks for the pass schedules.
 FwdPlan plan_forward_for(int64_t n, int64_t d, int64_t f, int P, tsp_dtype_t dt, tsp_sched_t sched,
                          size_t ws_bytes) {
     FwdPlan pl = plan_forward(n, d, f, P, dt, sched);
     if (pl.total() <= ws_bytes || dt != TSP_DT_BF16) return pl;
+    if (pl.fused) {
+        const size_t sync = align256(pl.sync_bytes);
+        if (ws_bytes <= sync + 256) {
+            pl.ok = false;
+            return pl;
+        }
+        pl = plan_forward_budget(n, d, f, P, dt, sched, ws_bytes - sync - 256);
+        if (pl.total() > ws_bytes) pl.ok = false;
+        return pl;
+    }
     const size_t acc = align256(static_cast<size_t>(n) * d * 4);
     if (ws_bytes <= acc + 256) {
         pl.ok = false;
@@ -422,7 +537,7 @@ tsp_status_t fwd_pass_bf16(const void* X, const void* Wg, const void* Wu, const 
     p1.width = static_cast<int>(width);
     p1.H = H;
     p1.ldh = width;
-    TSP_TRY(launch_umma<K1>(p1, st, dev, sms));
+    TSP_TRY(launch_pair<FwdHiddenPair<ACT>>(p1, st, dev, sms));
 
     typename K2::Params p2;
     std::memset(&p2, 0, sizeof(p2));
@@ -438,13 +553,70 @@ tsp_status_t fwd_pass_bf16(const void* X, const void* Wg, const void* Wu, const 
     p2.ldacc = d;
     p2.out = static_cast<__nv_bfloat16*>(Y);
     p2.ldo = d;
-    return launch_umma<K2>(p2, st, dev, sms);
+    return launch_pair<DownAccumPair<true, 1>>(p2, st, dev, sms);
+}
+
+// The whole forward as one persistent launch (fused.cuh).
+template <int ACT>
+tsp_status_t forward_bf16_fused(const void* X, const void* Wg, const void* Wu, const void* Wd,
+                                int64_t n, int64_t d, int64_t f, int P, const FwdPlan& pl,
+                                void* Y, void* ws, cudaStream_t st, int dev, int sms) {
+    using C = FusedFwd<ACT>;
+    char* w = static_cast<char*>(ws);
+    auto* H = reinterpret_cast<__nv_bfloat16*>(w);
+    auto* sync = reinterpret_cast<unsigned*>(w + align256(pl.ring_bytes));
+    FusedFwdParams p;
+    std::memset(&p, 0, sizeof(p));
+    if (!tmap_bf16(&p.tmX, X, d, n, d, 64, 128, SW128) ||
+        !tmap_bf16(&p.tmG, Wg, f, d, f, 64, 64, SW128) ||
+        (ACT == 1 && !tmap_bf16(&p.tmU, Wu, f, d, f, 64, 64, SW128)) ||
+        !tmap_bf16(&p.tmH, H, f, static_cast<uint64_t>(pl.R) * 128, f, 64, 128, SW128) ||
+        !tmap_bf16(&p.tmD, Wd, d, f, d, 64, 64, SW128))
+        return TSP_ERR_CUDA;
+    p.n = static_cast<int>(n);
+    p.d = static_cast<int>(d);
+    p.f = static_cast<int>(f);
+    p.seg_rows = pl.seg_rows;
+    p.mts = pl.mts;
+    p.ring = pl.ring ? 1 : 0;
+    p.fs = static_cast<int>(f / P);
+    p.MB = pl.MB;
+    p.nJ = static_cast<int>((f + C::kOut - 1) / C::kOut);
+    p.nC = static_cast<int>((d + 255) / 256);
+    p.GM = pl.GM;
+    p.G = (pl.MB + pl.GM - 1) / pl.GM;
+    p.head = sms;
+    p.R = pl.R;
+    p.total = p.MB * (p.nJ + p.nC);
+    p.H = H;
+    p.Y = static_cast<__nv_bfloat16*>(Y);
+    p.sync = sync;
+    if (cudaMemsetAsync(sync, 0, pl.sync_bytes, st) != cudaSuccess) return TSP_ERR_CUDA;
+    static bool attr_set[kMaxDevices] = {};
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!attr_set[dev]) {
+            if (cudaFuncSetAttribute(fused_mlp_fwd_kernel<ACT>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     C::kSmemBytes) != cudaSuccess)
+                return TSP_ERR_CUDA;
+            attr_set[dev] = true;
+        }
+    }
+    const int grid = std::min(p.total, sms);
+    TraceRec rec;
+    const bool traced = trace_begin(st, &rec, C::kName);
+    fused_mlp_fwd_kernel<ACT><<<grid, kPipelineThreads, C::kSmemBytes, st>>>(p);
+    const cudaError_t e = cudaGetLastError();
+    if (traced) trace_end(st, &rec);
+    return e == cudaSuccess ? TSP_OK : TSP_ERR_CUDA;
 }
 
 template <int ACT>
 tsp_status_t forward_bf16(const void* X, const void* Wg, const void* Wu, const void* Wd, int64_t n,
                           int64_t d, int64_t f, int P, const FwdPlan& pl, void* Y, void* ws,
                           cudaStream_t st, int dev, int sms) {
+    if (pl.fused) return forward_bf16_fused<ACT>(X, Wg, Wu, Wd, n, d, f, P, pl, Y, ws, st, dev, sms);
     auto* H = static_cast<__nv_bfloat16*>(ws);
     float* acc = pl.acc_bytes ? reinterpret_cast<float*>(static_cast<char*>(ws) +
                                                          align256(pl.h_bytes))
@@ -880,9 +1052,9 @@ tsp_status_t tsp_trace_reset(void) {
 tsp_status_t tsp_mlp_forward_noalloc(const void* X, const void* Wg, const void* Wu,
                                      const void* Wd, int64_t n, int64_t d, int64_t f, int P,
                                      tsp_act_t act, void* Y, tsp_stream_t stream) {
-    TSP_TRY(validate_forward(X, Wg, Wu, Wd, n, d, f, P, act, TSP_DT_BF16,
-                             TSP_SCHED_WEIGHT_SHARDS, Y));
-    const FwdPlan pl = plan_forward_for(n, d, f, P, TSP_DT_BF16, TSP_SCHED_WEIGHT_SHARDS,
+    // the fused schedule: its only scratch is the H ring and the counters
+    TSP_TRY(validate_forward(X, Wg, Wu, Wd, n, d, f, P, act, TSP_DT_BF16, TSP_SCHED_FUSED, Y));
+    const FwdPlan pl = plan_forward_for(n, d, f, P, TSP_DT_BF16, TSP_SCHED_FUSED,
                                         TSP_NOALLOC_SCRATCH_BYTES);
     if (!pl.ok || pl.total() > TSP_NOALLOC_SCRATCH_BYTES) return TSP_ERR_SCRATCH_LIMIT;
     int dev = 0;

@@ -47,21 +47,42 @@ def test_status_strings(lib):
     assert T.tsp_status_string(99) == "unknown status"
 
 
+def _a256(b):
+    return (b + 255) // 256 * 256
+
+
 def test_workspace_sizes_follow_the_schedule(lib):
     # fp32 weight-shard schedule: one shard's hidden block, Y accumulates in place
     assert T.tsp_mlp_workspace_size(64, 128, 512, 2, "gelu", "f32") == 64 * 256 * 4
-    # bf16, a single chunk: no fp32 accumulator is needed
-    assert T.tsp_mlp_workspace_size(256, 64, 512, 1, "swiglu", "bf16") == 256 * 512 * 2
-    # Llama-3-8B shape, P = 8: chunks of whole shards within the hidden budget
+    # bf16 fused schedule: an H ring of row-block slots (128 x d_ff) and the
+    # per-row-block counters; 2 row blocks -> 2 slots
+    assert T.tsp_mlp_workspace_size(256, 64, 512, 1, "swiglu", "bf16", "fused") == \
+        _a256(2 * 128 * 512 * 2) + _a256((1 + 2 * 2) * 4)
+    # Llama-3-8B shape: 32 row blocks in groups of 8, ring of 3 groups (24 slots)
     n, d, f, P = 4096, 4096, 14336, 8
-    ws = T.tsp_mlp_workspace_size(n, d, f, P, "swiglu", "bf16")
+    assert T.tsp_mlp_workspace_size(n, d, f, P, "swiglu", "bf16", "fused") == \
+        _a256(24 * 128 * f * 2) + _a256((1 + 2 * 32) * 4)
+    # pass schedule (also the default): chunks of whole shards within the hidden
+    # budget + the fp32 accumulator
+    ws = T.tsp_mlp_workspace_size(n, d, f, P, "swiglu", "bf16", "shard_passes")
+    assert ws == T.tsp_mlp_workspace_size(n, d, f, P, "swiglu", "bf16")
     acc = n * d * 4
     h = ws - acc
     assert h % (n * 2) == 0 and (h // (n * 2)) % (f // P) == 0
     assert h <= 64 << 20
-    # TSP ring: the hidden block of a group of sequence shards plus the accumulator
-    wsr = T.tsp_mlp_workspace_size(32768, d, f, P, "swiglu", "bf16", "tsp_ring")
-    assert wsr > acc * 8 and (wsr - 32768 * d * 4) % (4096 * (f // P) * 2) == 0
+    # single chunk: no accumulator
+    assert T.tsp_mlp_workspace_size(256, 64, 512, 1, "swiglu", "bf16", "shard_passes") == \
+        256 * 512 * 2
+    # TSP ring fused: 256 row blocks (8 sequence shards of 32), ring of 24 slots;
+    # TSP ring passes: sequence shards per launch within the hidden budget + accumulator
+    wsr = T.tsp_mlp_workspace_size(32768, d, f, P, "swiglu", "bf16", "tsp_ring_fused")
+    assert wsr == _a256(24 * 128 * f * 2) + _a256((1 + 2 * 256) * 4)
+    wsr2 = T.tsp_mlp_workspace_size(8 * 100, 256, 8 * 96, 8, "swiglu", "bf16", "tsp_ring")
+    assert wsr2 == _a256(8 * 100 * 96 * 2) + _a256(800 * 256 * 4)
+    # fused schedules need bf16; the fused ring needs 64-multiple shards
+    out = ctypes.c_size_t(0)
+    assert lib.tsp_mlp_workspace_size(64, 64, 128, 1, 1, 1, 3, 0, ctypes.byref(out)) == 2
+    assert lib.tsp_mlp_workspace_size(8 * 100, 256, 8 * 96, 8, 1, 0, 4, 0, ctypes.byref(out)) == 2
     # backward: H, dG, dU chunk buffers and the fp32 dX accumulator
     wsb = T.tsp_mlp_workspace_size(n, d, f, P, "swiglu", "bf16", backward=True)
     assert wsb > acc

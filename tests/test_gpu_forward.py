@@ -101,28 +101,46 @@ BF16_CASES = [
 ]
 
 
+@pytest.mark.parametrize("sched", ["weight_shards", "fused"])
 @pytest.mark.parametrize("act,n,d,f,P", BF16_CASES)
-def test_bf16_small_shapes(act, n, d, f, P):
+def test_bf16_small_shapes(act, n, d, f, P, sched):
     wl = small(act, "bf16", n, d, f, P, seed=n + d + f + P)
     inp = make_inputs(wl)
-    Y = gpu_forward(inp, P, act)
+    Y = gpu_forward(inp, P, act, sched)
     ref = oracle.mlp_forward(inp["X"], inp["A"], inp["Wu"], inp["B"], act)
     check(Y, ref, "bf16", wl.name)
 
 
 @pytest.mark.parametrize("act", ["swiglu", "gelu"])
 def test_bf16_multi_pass_accumulation(act):
-    """A workspace below the preferred size forces narrow hidden chunks, so the
-    fp32 accumulator goes through store, add and final passes."""
+    """The pass schedule with a workspace below its preferred size uses narrow
+    hidden chunks, so the fp32 accumulator goes through store, add and final
+    passes."""
     n, d, f, P = 384, 256, 8 * 192, 8
     wl = small(act, "bf16", n, d, f, P, seed=77)
     inp = make_inputs(wl)
     ws = n * d * 4 + 256 + n * 2 * 128 + 512   # one 128-column chunk + accumulator
-    Y = gpu_forward(inp, P, act, ws_bytes=ws)
+    Y = gpu_forward(inp, P, act, "shard_passes", ws_bytes=ws)
     ref = oracle.mlp_forward(inp["X"], inp["A"], inp["Wu"], inp["B"], act)
     check(Y, ref, "bf16", "multi-pass")
-    Y2 = gpu_forward(inp, P, act)  # preferred single pass agrees closely
+    Y2 = gpu_forward(inp, P, act)  # the fused schedule agrees closely
     assert np.abs(Y2 - Y).max() <= 2e-2 * np.abs(ref).max()
+
+
+@pytest.mark.parametrize("act", ["swiglu", "gelu"])
+def test_bf16_fused_small_ring_reuses_slots(act):
+    """A workspace with room for only three H-ring slots (groups of one row
+    block): every gate/up tile past the third row block waits for the down
+    tiles of the row block three earlier before overwriting its slot."""
+    n, d, f, P = 16 * 128 - 40, 256, 4 * 320, 4
+    wl = small(act, "bf16", n, d, f, P, seed=78)
+    inp = make_inputs(wl)
+    slot = 128 * f * 2
+    sync = (1 + 2 * 16) * 4
+    ws = 3 * slot + 256 + 512 + (sync + 255) // 256 * 256
+    Y = gpu_forward(inp, P, act, "fused", ws_bytes=ws)
+    ref = oracle.mlp_forward(inp["X"], inp["A"], inp["Wu"], inp["B"], act)
+    check(Y, ref, "bf16", "fused ring of 3 slots")
 
 
 @pytest.mark.parametrize("P", [1, 2, 4, 8])
@@ -134,21 +152,26 @@ def test_bf16_independent_of_P(P):
     check(Y, ref, "bf16", f"P={P}")
 
 
-@pytest.mark.parametrize("n,d,f,P", [(4 * 128, 128, 4 * 128, 4), (8 * 100, 256, 8 * 96, 8),
-                                     (2 * 64, 64, 2 * 64, 2)])
-def test_bf16_tsp_ring_small(n, d, f, P):
+@pytest.mark.parametrize("n,d,f,P,sched", [(4 * 128, 128, 4 * 128, 4, "tsp_ring"),
+                                           (8 * 100, 256, 8 * 96, 8, "tsp_ring"),
+                                           (2 * 64, 64, 2 * 64, 2, "tsp_ring"),
+                                           (4 * 128, 128, 4 * 128, 4, "tsp_ring_fused"),
+                                           (8 * 200, 256, 8 * 128, 8, "tsp_ring_fused"),
+                                           (2 * 64, 64, 2 * 64, 2, "tsp_ring_fused")])
+def test_bf16_tsp_ring_small(n, d, f, P, sched):
     wl = small("swiglu", "bf16", n, d, f, P, seed=11)
     inp = make_inputs(wl)
-    Y = gpu_forward(inp, P, "swiglu", "tsp_ring")
+    Y = gpu_forward(inp, P, "swiglu", sched)
     ref = oracle.mlp_tsp(inp["X"], inp["A"], inp["Wu"], inp["B"], "swiglu", P)
     check(Y, ref, "bf16", "tsp ring")
 
 
-def test_bf16_run_to_run_bitwise_deterministic():
-    wl = small("swiglu", "bf16", 640, 384, 8 * 128, 8, seed=21)
+@pytest.mark.parametrize("sched", ["weight_shards", "fused", "tsp_ring", "tsp_ring_fused"])
+def test_bf16_run_to_run_bitwise_deterministic(sched):
+    wl = small("swiglu", "bf16", 1024, 384, 8 * 128, 8, seed=21)
     inp = make_inputs(wl)
-    Y1 = gpu_forward(inp, 8, "swiglu", ws_bytes=640 * 384 * 4 + 640 * 2 * 256 + 4096)
-    Y2 = gpu_forward(inp, 8, "swiglu", ws_bytes=640 * 384 * 4 + 640 * 2 * 256 + 4096)
+    Y1 = gpu_forward(inp, 8, "swiglu", sched)
+    Y2 = gpu_forward(inp, 8, "swiglu", sched)
     assert np.array_equal(Y1, Y2)
 
 
@@ -189,19 +212,22 @@ def llama8b():
     return _full_inputs(LLAMA8B)
 
 
-@pytest.mark.parametrize("P", [8, 4, 2, 1])
-def test_llama8b_shape_sampled_rows(llama8b, P):
+@pytest.mark.parametrize("P,sched", [(8, "weight_shards"), (4, "weight_shards"),
+                                     (2, "weight_shards"), (1, "weight_shards"),
+                                     (8, "fused"), (1, "fused")])
+def test_llama8b_shape_sampled_rows(llama8b, P, sched):
     inp, dev = llama8b
-    Y = T.mlp_forward(dev["X"], dev["A"], dev["Wu"], dev["B"], P, "swiglu")
+    Y = T.mlp_forward(dev["X"], dev["A"], dev["Wu"], dev["B"], P, "swiglu", sched=sched)
     assert T.tsp_poll_device_error() == T.TSP_OK
     rows = sample_rows(LLAMA8B.n, 24, LLAMA8B.seed)
     _sampled_check(LLAMA8B, inp, Y, rows)
 
 
-def test_tsp_ring_long_context_sampled_rows():
+@pytest.mark.parametrize("sched", ["tsp_ring", "tsp_ring_fused"])
+def test_tsp_ring_long_context_sampled_rows(sched):
     inp, dev = _full_inputs(TSP_RING)
     Y = T.mlp_forward(dev["X"], dev["A"], dev["Wu"], dev["B"], TSP_RING.P, "swiglu",
-                      sched="tsp_ring")
+                      sched=sched)
     assert T.tsp_poll_device_error() == T.TSP_OK
     # rows from every sequence shard, including each shard's first and last row
     ns = TSP_RING.n // TSP_RING.P

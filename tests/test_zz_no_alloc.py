@@ -30,8 +30,8 @@ def _close(got, ref, what):
     assert np.linalg.norm(g - r) / np.linalg.norm(r) <= 5e-3, what
 
 
-# one case whose schedule needs several hidden chunks (fp32 accumulator in the
-# static array) and one that runs in a single chunk
+# one case whose hidden-activation ring in the static array holds fewer slots
+# than there are row blocks (slots are reused), and a small one
 CASES = [("swiglu", 2048, 2048, 14336, 8), ("gelu", 300, 520, 1024, 4)]
 
 
@@ -53,9 +53,9 @@ def test_noalloc_forward_matches_allocating_forward_twice(act, n, d, f, P):
 
 def test_noalloc_rejects_problems_beyond_its_static_scratch():
     T.load()
-    # n * d_model * 4 bytes of fp32 accumulator alone exceed the static array
+    # three hidden-activation slots of 128 x 65536 bf16 (48 MiB) exceed the array;
     # placeholder addresses far apart: the call returns before touching them
     X, A, U, B, Y = (k << 36 for k in range(1, 6))
-    s = T.tsp_mlp_forward_noalloc(X, A, U, B, 4096, 4096, 14336, 8, "swiglu", Y, check=False)
+    s = T.tsp_mlp_forward_noalloc(X, A, U, B, 4096, 4096, 65536, 8, "swiglu", Y, check=False)
     assert s == 7 and T.STATUS_NAMES[s] == "TSP_ERR_SCRATCH_LIMIT"
     assert "static" in T.tsp_status_string(s)
