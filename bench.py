@@ -241,7 +241,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=LLAMA8B.name, choices=sorted(WORKLOADS))
-    ap.add_argument("--sched", default=None, choices=["weight_shards", "tsp_ring", "shard_passes"],
+    ap.add_argument("--sched", default=None,
+                    choices=["weight_shards", "tsp_ring", "shard_passes", "fused", "tsp_ring_fused"],
                     help="override the workload's schedule")
     ap.add_argument("--ref-rows", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")

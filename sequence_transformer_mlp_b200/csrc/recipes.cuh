@@ -272,16 +272,21 @@ struct DownAccum {
         }
     }
     __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t acc, int q, int lane) {
-        const int rl = ti.mi * 128 + q * 32 + lane;
+        store_rows<8>(p, ti.s, ti.mi * 128 + q * 32 + lane, ti.nj * 256,
+                      acc + (static_cast<uint32_t>(q * 32) << 16));
+    }
+    // One thread's accumulator row (tile row rl of segment s) over NCHUNK x 32
+    // columns starting at output column col0, applied in the launch's mode.
+    template <int NCHUNK>
+    __device__ static void store_rows(const Params& p, int s, int rl, int col0, uint32_t t0) {
         const bool row_ok = rl < p.g.seg_rows;
-        const long long row = static_cast<long long>(p.g.seg_begin + ti.s) * p.g.seg_rows + rl;
-        const uint32_t t0 = acc + (static_cast<uint32_t>(q * 32) << 16);
+        const long long row = static_cast<long long>(p.g.seg_begin + s) * p.g.seg_rows + rl;
 #pragma unroll 1
-        for (int cc = 0; cc < 8; ++cc) {
+        for (int cc = 0; cc < NCHUNK; ++cc) {
             uint32_t v[32];
             tmem_ld_32x32b_x32(t0 + 32 * cc, v);
             tmem_ld_wait();
-            const int c0 = ti.nj * 256 + 32 * cc;
+            const int c0 = col0 + 32 * cc;
             const int valid = p.n_out - c0;
             if (!row_ok || valid <= 0) continue;
             if (p.mode == 0) {
@@ -331,148 +336,6 @@ struct DownAccum {
                         pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
                 }
                 store_bf16x32(p.out + row * p.ldo + c0, pk, valid);
-            }
-        }
-    }
-};
-
-// ============================================================================
-// K3: backward of the hidden layer for one column chunk.  Per tile (128 tokens
-// x 128 hidden columns) one pipeline computes, over K = d_model,
-//   G = X.W_gate[:, c..]  (and U = X.W_up[:, c..])   -- the recomputed forward
-//   dH = dY.W_down[c.., :]^T
-// and the epilogue emits H (for the W_down gradient) and the pre-activation
-// gradients: SwiGLU dU = dH SiLU(G), dG = dH U SiLU'(G); GeLU dG = dH GeLU'(G).
-// The pages only say the backward repeats the forward's pattern
-// ("Tensor Parallelism: Splitting the Math", the traffic count); the
-// derivatives are those of the forward definition.
-template <int ACT>
-struct BwdHidden {
-    struct Params {
-        CUtensorMap tmX;   // X  [n][d], box {32, 128}, 64B swizzle
-        CUtensorMap tmDY;  // dY [n][d], box {32, 128}, 64B swizzle
-        CUtensorMap tmG;   // W_gate / A [d][f], box {64, 32}
-        CUtensorMap tmU;   // W_up [d][f], box {64, 32} (SwiGLU)
-        CUtensorMap tmD;   // W_down / B [f][d], box {32, 128}, 64B swizzle
-        int n, d, col_base, width;
-        __nv_bfloat16 *H, *dG, *dU;  // [n][width]
-        long long ld;
-    };
-    static constexpr const char* kName = ACT == 1 ? "bwd_hidden_swiglu" : "bwd_hidden_gelu";
-    static constexpr int kBK = 32;
-    static constexpr int kTile = 8192;  // one 128 x 32 bf16 box
-    static constexpr int kOffX = 0, kOffDY = kTile, kOffG = 2 * kTile;
-    static constexpr int kOffU = 3 * kTile;
-    static constexpr int kOffD = ACT == 1 ? 4 * kTile : 3 * kTile;
-    static constexpr int kStageBytes = kOffD + kTile;
-    static constexpr int kStages = ACT == 1 ? 5 : 6;
-    static constexpr int kNGate = ACT == 1 ? 256 : 128;
-    static constexpr int kAccCols = ACT == 1 ? 512 : 256;
-    static constexpr int kAccBufs = ACT == 1 ? 1 : 2;
-    static constexpr int kTmemCols = 512;
-    static constexpr int kColDH = kNGate;  // TMEM column of dH
-    static constexpr uint32_t kIdesc1 = make_idesc_bf16(128, kNGate, false, true);
-    static constexpr uint32_t kIdesc2 = make_idesc_bf16(128, 128, false, false);
-    struct Tile {
-        int mi, nj;
-    };
-    __host__ __device__ static int num_tiles(const Params& p) {
-        return ((p.n + 127) / 128) * ((p.width + 127) / 128);
-    }
-    __device__ static Tile tile(const Params& p, int t) {
-        const int mt = (p.n + 127) / 128;
-        return Tile{t % mt, t / mt};
-    }
-    __device__ static int num_kb(const Params& p, const Tile&) { return (p.d + kBK - 1) / kBK; }
-    __device__ static void prefetch(const Params& p) {
-        tma_prefetch_desc(&p.tmX);
-        tma_prefetch_desc(&p.tmDY);
-        tma_prefetch_desc(&p.tmG);
-        if (ACT == 1) tma_prefetch_desc(&p.tmU);
-        tma_prefetch_desc(&p.tmD);
-    }
-    __device__ static uint32_t load_bytes(const Params&, const Tile&, int) { return kStageBytes; }
-    __device__ static void load(const Params& p, const Tile& ti, int kb, uint32_t st, uint32_t bar) {
-        const int k0 = kb * kBK;
-        const int r = ti.mi * 128;
-        const int c = p.col_base + ti.nj * 128;
-        tma_load_2d(st + kOffX, &p.tmX, bar, k0, r);
-        tma_load_2d(st + kOffDY, &p.tmDY, bar, k0, r);
-        tma_load_2d(st + kOffG, &p.tmG, bar, c, k0);
-        tma_load_2d(st + kOffG + 4096, &p.tmG, bar, c + 64, k0);
-        if (ACT == 1) {
-            tma_load_2d(st + kOffU, &p.tmU, bar, c, k0);
-            tma_load_2d(st + kOffU + 4096, &p.tmU, bar, c + 64, k0);
-        }
-        tma_load_2d(st + kOffD, &p.tmD, bar, k0, c);
-    }
-    __device__ static void mma(const Tile&, int kb, uint32_t st, uint32_t acc) {
-#pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint32_t en = (kb | kk) != 0 ? 1u : 0u;
-            const uint64_t ax = make_smem_desc(st + kOffX + 32 * kk, 16, 512, kLayoutSW64);
-            const uint64_t bg = make_smem_desc(st + kOffG + 2048 * kk, 4096, 1024, kLayoutSW128);
-            umma_bf16(acc, ax, bg, kIdesc1, en);
-            const uint64_t ady = make_smem_desc(st + kOffDY + 32 * kk, 16, 512, kLayoutSW64);
-            const uint64_t bd = make_smem_desc(st + kOffD + 32 * kk, 16, 512, kLayoutSW64);
-            umma_bf16(acc + kColDH, ady, bd, kIdesc2, en);
-        }
-    }
-    __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t acc, int q, int lane) {
-        const int row = ti.mi * 128 + q * 32 + lane;
-        const bool row_ok = row < p.n;
-        const long long off = static_cast<long long>(row) * p.ld;
-        const uint32_t t0 = acc + (static_cast<uint32_t>(q * 32) << 16);
-#pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-            uint32_t g[32], dh[32], ph[16], pg[16], pu[16];
-            tmem_ld_32x32b_x32(t0 + 32 * cc, g);
-            tmem_ld_32x32b_x32(t0 + kColDH + 32 * cc, dh);
-            if (ACT == 1) {
-                uint32_t u[32];
-                tmem_ld_32x32b_x32(t0 + 128 + 32 * cc, u);
-                tmem_ld_wait();
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    float hh[2], gg[2], uu[2];
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        const float gv = __uint_as_float(g[2 * i + j]);
-                        const float uv = __uint_as_float(u[2 * i + j]);
-                        const float dv = __uint_as_float(dh[2 * i + j]);
-                        const float sg = 1.0f / (1.0f + __expf(-gv));
-                        const float si = gv * sg;
-                        hh[j] = si * uv;
-                        uu[j] = dv * si;
-                        gg[j] = dv * uv * sg * (1.0f + gv * (1.0f - sg));
-                    }
-                    ph[i] = pack_bf16x2(hh[0], hh[1]);
-                    pg[i] = pack_bf16x2(gg[0], gg[1]);
-                    pu[i] = pack_bf16x2(uu[0], uu[1]);
-                }
-            } else {
-                tmem_ld_wait();
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    float hh[2], gg[2];
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        const float z = __uint_as_float(g[2 * i + j]);
-                        const float dv = __uint_as_float(dh[2 * i + j]);
-                        const float cdf = 0.5f * (1.0f + erff(z * 0.70710678118654752440f));
-                        const float pdf = 0.39894228040143267794f * __expf(-0.5f * z * z);
-                        hh[j] = z * cdf;
-                        gg[j] = dv * (cdf + z * pdf);
-                    }
-                    ph[i] = pack_bf16x2(hh[0], hh[1]);
-                    pg[i] = pack_bf16x2(gg[0], gg[1]);
-                }
-            }
-            const int c0 = ti.nj * 128 + 32 * cc;
-            if (row_ok) {
-                store_bf16x32(p.H + off + c0, ph, p.width - c0);
-                store_bf16x32(p.dG + off + c0, pg, p.width - c0);
-                if (ACT == 1) store_bf16x32(p.dU + off + c0, pu, p.width - c0);
             }
         }
     }

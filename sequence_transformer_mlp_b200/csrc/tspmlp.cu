@@ -33,7 +33,11 @@ constexpr int kMaxDevices = 64;
 // 126 MB L2 between the producing and the consuming kernel.
 constexpr size_t kFwdHiddenBudget = 64ull << 20;   // one bf16 [rows][C] buffer
 constexpr size_t kFusedRingBudget = 96ull << 20;   // the fused schedule's H ring
-constexpr size_t kBwdHiddenBudget = 96ull << 20;   // H, dG, dU together
+// H, dG, dU (bf16) and the fp32 activation-derivative factors together.  The
+// backward reads them from HBM anyway (the weight- and input-gradient kernels
+// run after the whole chunk is produced), so the chunk is sized for few, large
+// launches rather than for L2: one chunk at the Llama-3-8B shape.
+constexpr size_t kBwdHiddenBudget = 1024ull << 20;
 
 struct DevInfo {
     bool probed = false;
@@ -553,7 +557,7 @@ tsp_status_t fwd_pass_bf16(const void* X, const void* Wg, const void* Wu, const 
     p2.ldacc = d;
     p2.out = static_cast<__nv_bfloat16*>(Y);
     p2.ldo = d;
-    return launch_pair<DownAccumPair<true, 1>>(p2, st, dev, sms);
+    return launch_pair<DownAccumPair<true, 1, 256>>(p2, st, dev, sms);
 }
 
 // The whole forward as one persistent launch (fused.cuh).
@@ -686,16 +690,20 @@ tsp_status_t forward_f32(const float* X, const float* Wg, const float* Wu, const
 struct BwdPlan {
     bool ok = true;
     std::vector<Chunk> chunks;
-    size_t buf_bytes = 0;  // one of H / dG / dU
-    int nbufs = 3;
+    int n16 = 3, n32 = 2;     // bf16 buffers (H, dG, dU) and fp32 factor buffers (S1, S2)
+    size_t b16 = 0, b32 = 0;  // bytes of one bf16 / fp32 chunk buffer
     size_t acc_bytes = 0;
-    size_t total() const { return nbufs * align256(buf_bytes) + align256(acc_bytes); }
+    size_t total() const {
+        return n16 * align256(b16) + n32 * align256(b32) + align256(acc_bytes);
+    }
 };
 
 BwdPlan plan_backward_budget(int64_t n, int64_t d, int64_t f, int P, tsp_act_t act, size_t budget) {
     BwdPlan pl;
-    pl.nbufs = act == TSP_ACT_SWIGLU ? 3 : 2;
-    const int64_t mc = max_chunk_cols(budget, static_cast<size_t>(n) * 2 * pl.nbufs);
+    pl.n16 = act == TSP_ACT_SWIGLU ? 3 : 2;
+    pl.n32 = act == TSP_ACT_SWIGLU ? 2 : 1;
+    const size_t per_col = static_cast<size_t>(n) * (2 * pl.n16 + 4 * pl.n32);
+    const int64_t mc = max_chunk_cols(budget, per_col);
     if (mc == 0) {
         pl.ok = false;
         return pl;
@@ -703,7 +711,8 @@ BwdPlan plan_backward_budget(int64_t n, int64_t d, int64_t f, int P, tsp_act_t a
     pl.chunks = plan_chunks(f, P, mc);
     int64_t wmax = 0;
     for (auto& c : pl.chunks) wmax = std::max(wmax, c.width);
-    pl.buf_bytes = static_cast<size_t>(n) * wmax * 2;
+    pl.b16 = static_cast<size_t>(n) * wmax * 2;
+    pl.b32 = static_cast<size_t>(n) * wmax * 4;
     pl.acc_bytes = pl.chunks.size() > 1 ? static_cast<size_t>(n) * d * 4 : 0;
     return pl;
 }
@@ -716,11 +725,11 @@ BwdPlan plan_backward_for(int64_t n, int64_t d, int64_t f, int P, tsp_act_t act,
     BwdPlan pl = plan_backward(n, d, f, P, act);
     if (pl.total() <= ws_bytes) return pl;
     const size_t acc = align256(static_cast<size_t>(n) * d * 4);
-    if (ws_bytes <= acc + 1024) {
+    if (ws_bytes <= acc + 2048) {
         pl.ok = false;
         return pl;
     }
-    pl = plan_backward_budget(n, d, f, P, act, ws_bytes - acc - 1024);
+    pl = plan_backward_budget(n, d, f, P, act, ws_bytes - acc - 2048);
     if (pl.total() > ws_bytes) pl.ok = false;
     return pl;
 }
@@ -731,35 +740,52 @@ tsp_status_t backward_bf16(const void* X, const void* Wg, const void* Wu, const 
                            const BwdPlan& pl, void* dX, float* dWg, float* dWu, float* dWd,
                            void* ws, cudaStream_t st, int dev, int sms) {
     char* w = static_cast<char*>(ws);
-    const size_t bb = align256(pl.buf_bytes);
+    const size_t a16 = align256(pl.b16), a32 = align256(pl.b32);
     auto* Hc = reinterpret_cast<__nv_bfloat16*>(w);
-    auto* dGc = reinterpret_cast<__nv_bfloat16*>(w + bb);
-    auto* dUc = ACT == 1 ? reinterpret_cast<__nv_bfloat16*>(w + 2 * bb) : nullptr;
-    float* acc = pl.acc_bytes ? reinterpret_cast<float*>(w + pl.nbufs * bb) : nullptr;
+    auto* dGc = reinterpret_cast<__nv_bfloat16*>(w + a16);
+    auto* dUc = ACT == 1 ? reinterpret_cast<__nv_bfloat16*>(w + 2 * a16) : nullptr;
+    auto* S1 = reinterpret_cast<float*>(w + pl.n16 * a16);
+    auto* S2 = ACT == 1 ? reinterpret_cast<float*>(w + pl.n16 * a16 + a32) : nullptr;
+    float* acc = pl.acc_bytes ? reinterpret_cast<float*>(w + pl.n16 * a16 + pl.n32 * a32) : nullptr;
     const int64_t fs = f / P;
     const int np = static_cast<int>(pl.chunks.size());
     for (int i = 0; i < np; ++i) {
         const int64_t cb = pl.chunks[i].col_base, C = pl.chunks[i].width;
-        // K3: recompute G (U), dH; emit H, dG (dU)
+        // K3a: recompute G (U); emit H and the activation-derivative factors
         {
-            using K = BwdHidden<ACT>;
-            typename K::Params p;
+            BwdGateUpParams p;
             std::memset(&p, 0, sizeof(p));
-            if (!tmap_bf16(&p.tmX, X, d, n, d, 32, 128, SW64) ||
-                !tmap_bf16(&p.tmDY, dY, d, n, d, 32, 128, SW64) ||
-                !tmap_bf16(&p.tmG, Wg, f, d, f, 64, 32, SW128) ||
-                (ACT == 1 && !tmap_bf16(&p.tmU, Wu, f, d, f, 64, 32, SW128)) ||
-                !tmap_bf16(&p.tmD, Wd, d, f, d, 32, 128, SW64))
+            if (!tmap_bf16(&p.tmX, X, d, n, d, 64, 128, SW128) ||
+                !tmap_bf16(&p.tmG, Wg, f, d, f, 64, 64, SW128) ||
+                (ACT == 1 && !tmap_bf16(&p.tmU, Wu, f, d, f, 64, 64, SW128)))
                 return TSP_ERR_CUDA;
             p.n = static_cast<int>(n);
             p.d = static_cast<int>(d);
             p.col_base = static_cast<int>(cb);
             p.width = static_cast<int>(C);
             p.H = Hc;
+            p.S1 = S1;
+            p.S2 = S2;
+            p.ld = C;
+            TSP_TRY(launch_pair<BwdGateUpPair<ACT>>(p, st, dev, sms));
+        }
+        // K3b: dH = dY . W_down[chunk]^T; emit dG (dU) from the factors
+        {
+            DhParams p;
+            std::memset(&p, 0, sizeof(p));
+            if (!tmap_bf16(&p.tmDY, dY, d, n, d, 64, 128, SW128) ||
+                !tmap_bf16(&p.tmD, Wd, d, f, d, 64, 128, SW128))
+                return TSP_ERR_CUDA;
+            p.n = static_cast<int>(n);
+            p.d = static_cast<int>(d);
+            p.col_base = static_cast<int>(cb);
+            p.width = static_cast<int>(C);
+            p.S1 = S1;
+            p.S2 = S2;
             p.dG = dGc;
             p.dU = dUc;
             p.ld = C;
-            TSP_TRY(launch_umma<K>(p, st, dev, sms));
+            TSP_TRY(launch_pair<DhPair<ACT>>(p, st, dev, sms));
         }
         // K4a: dW_down[cb .. cb+C) = H^T . dY
         {
@@ -776,7 +802,7 @@ tsp_status_t backward_bf16(const void* X, const void* Wg, const void* Wu, const 
             p.ldo = d;
             p.out_row0 = static_cast<int>(cb);
             p.out_col0 = 0;
-            TSP_TRY(launch_umma<K>(p, st, dev, sms));
+            TSP_TRY((launch_pair<WgradPair<256, false>>(p, st, dev, sms)));
         }
         // K4b: dW_gate (dW_up)[:, cb .. cb+C) = X^T . dG (dU)
         if (ACT == 1) {
@@ -795,7 +821,7 @@ tsp_status_t backward_bf16(const void* X, const void* Wg, const void* Wu, const 
             p.ldo = f;
             p.out_row0 = 0;
             p.out_col0 = static_cast<int>(cb);
-            TSP_TRY(launch_umma<K>(p, st, dev, sms));
+            TSP_TRY((launch_pair<WgradPair<256, true>>(p, st, dev, sms)));
         } else {
             using K = Wgrad<128, false>;
             typename K::Params p;
@@ -810,20 +836,22 @@ tsp_status_t backward_bf16(const void* X, const void* Wg, const void* Wu, const 
             p.ldo = f;
             p.out_row0 = 0;
             p.out_col0 = static_cast<int>(cb);
-            TSP_TRY(launch_umma<K>(p, st, dev, sms));
+            TSP_TRY((launch_pair<WgradPair<128, false>>(p, st, dev, sms)));
         }
         // K5: dX (+)= dG . W_gate[:, chunk]^T (+ dU . W_up[:, chunk]^T)
         {
-            using K = DownAccum<false, ACT == 1 ? 2 : 1>;
+            constexpr int NS = ACT == 1 ? 2 : 1;
+            using K = DownAccum<false, NS>;
             typename K::Params p;
             std::memset(&p, 0, sizeof(p));
+            p.g = seg_all_rows(n, P, fs, cb);
+            p.n_out = static_cast<int>(d);
             if (!tmap_bf16(&p.tmA0, dGc, C, n, C, 64, 128, SW128) ||
-                !tmap_bf16(&p.tmB0, Wg, f, d, f, 64, 256, SW128))
+                !tmap_bf16(&p.tmB0, Wg, f, d, f, 64, 128, SW128))
                 return TSP_ERR_CUDA;
             if (ACT == 1 && (!tmap_bf16(&p.tmA1, dUc, C, n, C, 64, 128, SW128) ||
-                             !tmap_bf16(&p.tmB1, Wu, f, d, f, 64, 256, SW128)))
+                             !tmap_bf16(&p.tmB1, Wu, f, d, f, 64, 128, SW128)))
                 return TSP_ERR_CUDA;
-            p.g = seg_all_rows(n, P, fs, cb);
             p.kdim = static_cast<int>(C);
             p.n_out = static_cast<int>(d);
             p.mode = accum_mode(i, np);
@@ -831,7 +859,7 @@ tsp_status_t backward_bf16(const void* X, const void* Wg, const void* Wu, const 
             p.ldacc = d;
             p.out = static_cast<__nv_bfloat16*>(dX);
             p.ldo = d;
-            TSP_TRY(launch_umma<K>(p, st, dev, sms));
+            TSP_TRY((launch_pair<DownAccumPair<false, NS, 256>>(p, st, dev, sms)));
         }
     }
     return TSP_OK;
