@@ -41,7 +41,7 @@ sys.path.insert(0, ROOT)
 from workloads import WORKLOADS, LLAMA8B, make_inputs  # noqa: E402
 
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
-KERNEL_SOURCES = ["ptx.cuh", "pipeline.cuh", "recipes.cuh"]
+KERNEL_SOURCES = ["ptx.cuh", "pipeline.cuh", "pipeline2.cuh", "recipes.cuh", "fused.cuh", "fused2.cuh"]
 
 
 def peaks():
@@ -209,29 +209,51 @@ def replica_throughput(world: int, flops_per_step: float, ms_max: float) -> floa
 
 
 def end_to_end(args, inp, dev, step, Y, stream, barrier):
-    """The same step through the public call with host buffers: every step
-    copies X in from pinned host memory and reads Y back, all inside the
-    timed region.  Returns (ms per step, host X, host Y)."""
+    """The same step through the public call with host buffers, pipelined as a
+    serving loop would run it: every step copies its X in from pinned host
+    memory (copy-in stream) and reads its Y back (copy-out stream), and the
+    copies of neighbouring steps overlap the compute of the current one
+    (device X and Y double-buffered, ordered with events).  All copies are
+    inside the timed region.  Returns (ms per step, host X, host Y)."""
     n, d = inp["X"].shape
     Xh = inp["X"].pin_memory()
-    Yh = torch.empty(n, d, dtype=torch.bfloat16).pin_memory()
-    Xd = torch.empty_like(dev["X"])
-    for _ in range(2):
-        Xd.copy_(Xh, non_blocking=True)
-        step(Xd)
-        Yh.copy_(Y, non_blocking=True)
+    Yh = [torch.empty(n, d, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    Xd = [torch.empty_like(dev["X"]) for _ in range(2)]
+    Yd = [torch.empty_like(Y) for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()
+    in_done, comp_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+
+    def run(k):
+        for i in range(k):
+            b = i & 1
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(comp_done[b])      # X[b] of step i-2 consumed
+                Xd[b].copy_(Xh, non_blocking=True)
+                in_done[b].record(s_in)
+            stream.wait_event(in_done[b])
+            if i >= 2:
+                stream.wait_event(out_done[b])         # Y[b] of step i-2 read back
+            step(Xd[b], Yd[b])
+            comp_done[b].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(comp_done[b])
+                Yh[b].copy_(Yd[b], non_blocking=True)
+                out_done[b].record(s_out)
+
+    run(4)
     torch.cuda.synchronize()
     barrier()
     e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e2.record(stream)
-    for _ in range(args.steps):
-        Xd.copy_(Xh, non_blocking=True)
-        step(Xd)
-        Yh.copy_(Y, non_blocking=True)
-    e3.record(stream)
+    e2.record(s_in)
+    run(args.steps)
+    s_out.wait_stream(s_in)
+    s_out.wait_stream(stream)
+    e3.record(s_out)
     torch.cuda.synchronize()
     barrier()
-    return e2.elapsed_time(e3) / args.steps, Xh, Yh
+    return e2.elapsed_time(e3) / args.steps, Xh, Yh[0]
 
 
 def main():
@@ -242,7 +264,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=LLAMA8B.name, choices=sorted(WORKLOADS))
     ap.add_argument("--sched", default=None,
-                    choices=["weight_shards", "tsp_ring", "shard_passes", "fused", "tsp_ring_fused"],
+                    choices=["weight_shards", "tsp_ring", "shard_passes", "fused", "tsp_ring_fused",
+                             "shard_passes_fused"],
                     help="override the workload's schedule")
     ap.add_argument("--ref-rows", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -289,9 +312,9 @@ def main():
         ws_f = torch.empty(max(T.tsp_mlp_workspace_size(n, d, f, P, wl.act, "bf16", sched), 1),
                            dtype=torch.uint8, device="cuda")
 
-    def step(x=dev["X"]):
+    def step(x=dev["X"], y=Y):
         T.tsp_mlp_forward_ex(x, dev["A"], dev["Wu"], dev["B"], n, d, f, P, wl.act, "bf16", sched,
-                             Y, ws_f if wl.backward else ws,
+                             y, ws_f if wl.backward else ws,
                              ws_f.numel() if wl.backward else need, stream)
         if wl.backward:
             T.tsp_mlp_backward_ex(x, dev["A"], dev["Wu"], dev["B"], dev["dY"], n, d, f, P, wl.act,
@@ -388,8 +411,8 @@ def kernel_flops_per_step(kernel: str, wl) -> float:
     product it computes).  Per step the forward hidden kernel covers all n x f
     hidden units once and the down kernel all n x d outputs over K = d_ff,
     whatever the number of launches (chunks, ring steps) they are split into.
-    The backward hidden kernel's recomputed G/U products are counted: they run
-    on the tensor cores like the rest."""
+    The backward's recomputed gate/up products are counted: they run on the
+    tensor cores like the rest."""
     n, d, f = wl.n, wl.d, wl.f
     return {
         "fused_fwd_swiglu": 2 * 3 * n * d * f,
@@ -397,8 +420,12 @@ def kernel_flops_per_step(kernel: str, wl) -> float:
         "fwd_hidden_swiglu": 2 * 2 * n * d * f,
         "fwd_hidden_gelu": 2 * n * d * f,
         "down_accum_fwd": 2 * n * d * f,
-        "bwd_hidden_swiglu": 2 * 3 * n * d * f,
-        "bwd_hidden_gelu": 2 * 2 * n * d * f,
+        "fused_passes_swiglu": 2 * 3 * n * d * f,
+        "fused_passes_gelu": 2 * 2 * n * d * f,
+        "bwd_gate_up_swiglu": 2 * 2 * n * d * f,
+        "bwd_gate_up_gelu": 2 * n * d * f,
+        "bwd_dh_swiglu": 2 * n * d * f,
+        "bwd_dh_gelu": 2 * n * d * f,
         "wgrad_down": 2 * n * d * f,
         "wgrad_gate_up": 2 * 2 * n * d * f,
         "wgrad_gelu_a": 2 * n * d * f,

@@ -85,7 +85,7 @@ typedef enum { TSP_DT_BF16 = 0, TSP_DT_F32 = 1 } tsp_dtype_t;
 typedef enum {
     /* Weight-shard schedule: every token meets shard 0, 1, ..., P-1 in order
      * and the partial outputs accumulate in that order (the library picks its
-     * fastest implementation; today TSP_SCHED_SHARD_PASSES for bf16). */
+     * fastest measured implementation: TSP_SCHED_SHARD_PASSES for bf16). */
     TSP_SCHED_WEIGHT_SHARDS = 0,
     /* Folded tensor-and-sequence ring: tokens form P equal sequence shards;
      * at ring step t sequence shard s meets weight shard (s + t) mod P and
@@ -104,7 +104,12 @@ typedef enum {
     /* The TSP ring as one persistent launch (bf16): as TSP_SCHED_FUSED, each
      * sequence shard's K loop over the hidden units starting at its own weight
      * shard.  Needs n % P == 0 and (d_ff / P) % 64 == 0. */
-    TSP_SCHED_TSP_RING_FUSED = 4
+    TSP_SCHED_TSP_RING_FUSED = 4,
+    /* TSP_SCHED_SHARD_PASSES with all passes in one persistent launch on CTA
+     * pairs (bf16): chunk c's down-projection tiles run alongside chunk c+1's
+     * gate/up tiles, ordered by per-row-block counters.  Needs
+     * (d_ff / P) % 64 == 0 and at most 32 chunks. */
+    TSP_SCHED_SHARD_PASSES_FUSED = 5
 } tsp_sched_t;
 
 /* Forward pass, bf16, weight-shard schedule.

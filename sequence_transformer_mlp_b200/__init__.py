@@ -36,7 +36,7 @@ NOALLOC_SCRATCH_BYTES = 32 << 20
 ACT = {"gelu": 0, "swiglu": 1}
 DTYPE = {"bf16": 0, "f32": 1}
 SCHED = {"weight_shards": 0, "tsp_ring": 1, "shard_passes": 2, "fused": 3,
-         "tsp_ring_fused": 4}
+         "tsp_ring_fused": 4, "shard_passes_fused": 5}
 
 
 class KernelStat(ctypes.Structure):

@@ -20,6 +20,7 @@
 
 #include "../../include/tspmlp.h"
 #include "fused.cuh"
+#include "fused2.cuh"
 #include "pipeline2.cuh"
 #include "recipes.cuh"
 #include "simt_f32.cuh"
@@ -33,6 +34,7 @@ constexpr int kMaxDevices = 64;
 // 126 MB L2 between the producing and the consuming kernel.
 constexpr size_t kFwdHiddenBudget = 64ull << 20;   // one bf16 [rows][C] buffer
 constexpr size_t kFusedRingBudget = 96ull << 20;   // the fused schedule's H ring
+constexpr size_t kFusedPassesBudget = 128ull << 20; // two H chunk buffers of the one-launch passes
 // H, dG, dU (bf16) and the fp32 activation-derivative factors together.  The
 // backward reads them from HBM anyway (the weight- and input-gradient kernels
 // run after the whole chunk is produced), so the chunk is sized for few, large
@@ -301,15 +303,18 @@ tsp_status_t validate_shape(int64_t n, int64_t d, int64_t f, int P, tsp_act_t ac
                             tsp_dtype_t dt, tsp_sched_t sched) {
     if (act != TSP_ACT_GELU && act != TSP_ACT_SWIGLU) return TSP_ERR_INVALID_ARG;
     if (dt != TSP_DT_BF16 && dt != TSP_DT_F32) return TSP_ERR_INVALID_ARG;
-    if (sched < TSP_SCHED_WEIGHT_SHARDS || sched > TSP_SCHED_TSP_RING_FUSED)
+    if (sched < TSP_SCHED_WEIGHT_SHARDS || sched > TSP_SCHED_SHARD_PASSES_FUSED)
         return TSP_ERR_INVALID_ARG;
     if (n <= 0 || d <= 0 || f <= 0 || P <= 0) return TSP_ERR_INVALID_ARG;
     if (n > kMaxDim || d > kMaxDim || f > kMaxDim || P > 4096) return TSP_ERR_UNSUPPORTED_SHAPE;
     if (f % P != 0) return TSP_ERR_UNSUPPORTED_SHAPE;
     const bool ring = sched == TSP_SCHED_TSP_RING || sched == TSP_SCHED_TSP_RING_FUSED;
     if (ring && n % P != 0) return TSP_ERR_UNSUPPORTED_SHAPE;
-    if ((sched == TSP_SCHED_FUSED || sched == TSP_SCHED_TSP_RING_FUSED) && dt != TSP_DT_BF16)
+    if ((sched == TSP_SCHED_FUSED || sched == TSP_SCHED_TSP_RING_FUSED ||
+         sched == TSP_SCHED_SHARD_PASSES_FUSED) &&
+        dt != TSP_DT_BF16)
         return TSP_ERR_UNSUPPORTED_SHAPE;
+    if (sched == TSP_SCHED_SHARD_PASSES_FUSED && (f / P) % 64 != 0) return TSP_ERR_UNSUPPORTED_SHAPE;
     if (sched == TSP_SCHED_TSP_RING_FUSED && (f / P) % 64 != 0) return TSP_ERR_UNSUPPORTED_SHAPE;
     if (dt == TSP_DT_BF16 && (d % 8 != 0 || (f / P) % 8 != 0)) return TSP_ERR_UNSUPPORTED_SHAPE;
     return TSP_OK;
@@ -376,6 +381,8 @@ tsp_status_t validate_backward(const void* X, const void* Wg, const void* Wu, co
 struct FwdPlan {
     bool ok = true;
     bool ring = false;
+    // the pass schedule in one paired launch (two H chunk buffers)
+    bool fused_passes = false;
     // fused single-launch schedule (bf16)
     bool fused = false;
     int segs = 1, seg_rows = 0, mts = 0, MB = 0, GM = 1, R = 1;
@@ -385,8 +392,9 @@ struct FwdPlan {
     int tsp_group = 1;          // ring passes: sequence shards per launch
     size_t h_bytes = 0, acc_bytes = 0;
     size_t total() const {
-        return fused ? align256(ring_bytes) + align256(sync_bytes)
-                     : align256(h_bytes) + align256(acc_bytes);
+        if (fused) return align256(ring_bytes) + align256(sync_bytes);
+        if (fused_passes) return 2 * align256(h_bytes) + align256(acc_bytes) + align256(sync_bytes);
+        return align256(h_bytes) + align256(acc_bytes);
     }
 };
 
@@ -445,12 +453,20 @@ FwdPlan plan_forward_budget(int64_t n, int64_t d, int64_t f, int P, tsp_dtype_t 
         return pl;
     }
     if (dt == TSP_DT_BF16) {
-        const int64_t mc = max_chunk_cols(budget, static_cast<size_t>(n) * 2);
+        // the one-launch pass schedule holds two H chunks; it needs chunk widths
+        // that are whole 64-column k-blocks and at most kFusedMaxChunks chunks
+        const bool try_fused = sched == TSP_SCHED_SHARD_PASSES_FUSED;
+        const int64_t mc = max_chunk_cols(try_fused ? budget / 2 : budget, static_cast<size_t>(n) * 2);
         if (mc == 0) {
             pl.ok = false;
             return pl;
         }
         pl.chunks = plan_chunks(f, P, mc);
+        if (try_fused) {
+            pl.fused_passes = true;
+            pl.ok = static_cast<int>(pl.chunks.size()) <= kFusedMaxChunks;
+            pl.sync_bytes = static_cast<size_t>(1 + 2 * pl.chunks.size() * ((n + 255) / 256)) * 4;
+        }
     } else {
         for (int w = 0; w < P; ++w) pl.chunks.push_back({w * fs, fs});
     }
@@ -465,7 +481,9 @@ FwdPlan plan_forward_budget(int64_t n, int64_t d, int64_t f, int P, tsp_dtype_t 
 FwdPlan plan_forward(int64_t n, int64_t d, int64_t f, int P, tsp_dtype_t dt, tsp_sched_t sched) {
     FwdPlan pl = plan_forward_budget(n, d, f, P, dt, sched, kFusedRingBudget);
     if (pl.fused) return pl;
-    return plan_forward_budget(n, d, f, P, dt, sched, kFwdHiddenBudget);
+    return plan_forward_budget(n, d, f, P, dt, sched,
+                               sched == TSP_SCHED_SHARD_PASSES_FUSED ? kFusedPassesBudget
+                                                                     : kFwdHiddenBudget);
 }
 
 // The schedule for a caller workspace of ws_bytes: the preferred one if it
@@ -486,6 +504,18 @@ FwdPlan plan_forward_for(int64_t n, int64_t d, int64_t f, int P, tsp_dtype_t dt,
         return pl;
     }
     const size_t acc = align256(static_cast<size_t>(n) * d * 4);
+    if (sched == TSP_SCHED_SHARD_PASSES_FUSED) {
+        // two H chunk buffers and the counters
+        const size_t sync =
+            align256(static_cast<size_t>(1 + 2 * kFusedMaxChunks * ((n + 255) / 256)) * 4);
+        if (ws_bytes <= acc + sync + 512) {
+            pl.ok = false;
+            return pl;
+        }
+        pl = plan_forward_budget(n, d, f, P, dt, sched, ws_bytes - acc - sync - 512);
+        if (pl.total() > ws_bytes) pl.ok = false;
+        return pl;
+    }
     if (ws_bytes <= acc + 256) {
         pl.ok = false;
         return pl;
@@ -616,11 +646,104 @@ tsp_status_t forward_bf16_fused(const void* X, const void* Wg, const void* Wu, c
     return e == cudaSuccess ? TSP_OK : TSP_ERR_CUDA;
 }
 
+// The pass schedule as one persistent paired launch (fused2.cuh).
+template <int ACT>
+tsp_status_t forward_bf16_fused_passes(const void* X, const void* Wg, const void* Wu,
+                                       const void* Wd, int64_t n, int64_t d, int64_t f,
+                                       const FwdPlan& pl, void* Y, void* ws, cudaStream_t st,
+                                       int dev, int sms) {
+    using Cfg = FusedPassesCfg<ACT>;
+    char* w = static_cast<char*>(ws);
+    const size_t hb = align256(pl.h_bytes);
+    int64_t wmax = 0;
+    for (auto& c : pl.chunks) wmax = std::max(wmax, c.width);
+    auto* H0 = reinterpret_cast<__nv_bfloat16*>(w);
+    auto* H1 = reinterpret_cast<__nv_bfloat16*>(w + hb);
+    float* acc = pl.acc_bytes ? reinterpret_cast<float*>(w + 2 * hb) : nullptr;
+    auto* sync = reinterpret_cast<unsigned*>(w + 2 * hb + align256(pl.acc_bytes));
+    FusedPassesParams p;
+    std::memset(&p, 0, sizeof(p));
+    if (!tmap_bf16(&p.tmX, X, d, n, d, 64, 128, SW128) ||
+        !tmap_bf16(&p.tmG, Wg, f, d, f, 64, 64, SW128) ||
+        (ACT == 1 && !tmap_bf16(&p.tmU, Wu, f, d, f, 64, 64, SW128)) ||
+        !tmap_bf16(&p.tmH0, H0, wmax, n, wmax, 64, 128, SW128) ||
+        !tmap_bf16(&p.tmH1, H1, wmax, n, wmax, 64, 128, SW128) ||
+        !tmap_bf16(&p.tmD, Wd, d, f, d, 64, 64, SW128))
+        return TSP_ERR_CUDA;
+    p.n = static_cast<int>(n);
+    p.d = static_cast<int>(d);
+    p.f = static_cast<int>(f);
+    p.MP = static_cast<int>((n + 255) / 256);
+    p.C = static_cast<int>(pl.chunks.size());
+    for (int i = 0; i < p.C; ++i) {
+        p.cb[i] = static_cast<int>(pl.chunks[i].col_base);
+        p.cw[i] = static_cast<int>(pl.chunks[i].width);
+    }
+    p.nN = static_cast<int>((d + 255) / 256);
+    p.wmax = static_cast<int>(wmax);
+    p.H0 = H0;
+    p.H1 = H1;
+    p.acc = acc;
+    p.Y = static_cast<__nv_bfloat16*>(Y);
+    p.sync = sync;
+    int total = 0;
+    for (int i = 0; i < p.C; ++i) total += pass_nj<Cfg::kOut>(p, i) * p.MP + p.nN * p.MP;
+    p.total = total;
+    const size_t sync_bytes = static_cast<size_t>(1 + 2 * p.C * p.MP) * 4;
+    if (cudaMemsetAsync(sync, 0, sync_bytes, st) != cudaSuccess) return TSP_ERR_CUDA;
+    static bool attr_set[kMaxDevices] = {};
+    static int max_pairs[kMaxDevices] = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!attr_set[dev]) {
+            if (cudaFuncSetAttribute(fused_passes_pair_kernel<ACT>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     Cfg::kSmemBytes) != cudaSuccess)
+                return TSP_ERR_CUDA;
+            cudaLaunchConfig_t q = {};
+            q.gridDim = dim3(static_cast<unsigned>(sms / 2 * 2));
+            q.blockDim = dim3(kPipelineThreads);
+            q.dynamicSmemBytes = Cfg::kSmemBytes;
+            q.attrs = attr;
+            q.numAttrs = 1;
+            int nc = 0;
+            if (cudaOccupancyMaxActiveClusters(&nc, fused_passes_pair_kernel<ACT>, &q) != cudaSuccess ||
+                nc <= 0) {
+                cudaGetLastError();
+                nc = sms / 2;
+            }
+            max_pairs[dev] = nc;
+            attr_set[dev] = true;
+        }
+    }
+    const int pairs = std::min(total, max_pairs[dev]);
+    p.head = pairs;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+    cfg.blockDim = dim3(kPipelineThreads);
+    cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    TraceRec rec;
+    const bool traced = trace_begin(st, &rec, Cfg::kName);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, fused_passes_pair_kernel<ACT>, p);
+    if (traced) trace_end(st, &rec);
+    return e == cudaSuccess ? TSP_OK : TSP_ERR_CUDA;
+}
+
 template <int ACT>
 tsp_status_t forward_bf16(const void* X, const void* Wg, const void* Wu, const void* Wd, int64_t n,
                           int64_t d, int64_t f, int P, const FwdPlan& pl, void* Y, void* ws,
                           cudaStream_t st, int dev, int sms) {
     if (pl.fused) return forward_bf16_fused<ACT>(X, Wg, Wu, Wd, n, d, f, P, pl, Y, ws, st, dev, sms);
+    if (pl.fused_passes)
+        return forward_bf16_fused_passes<ACT>(X, Wg, Wu, Wd, n, d, f, pl, Y, ws, st, dev, sms);
     auto* H = static_cast<__nv_bfloat16*>(ws);
     float* acc = pl.acc_bytes ? reinterpret_cast<float*>(static_cast<char*>(ws) +
                                                          align256(pl.h_bytes))

@@ -62,11 +62,14 @@ def test_workspace_sizes_follow_the_schedule(lib):
     n, d, f, P = 4096, 4096, 14336, 8
     assert T.tsp_mlp_workspace_size(n, d, f, P, "swiglu", "bf16", "fused") == \
         _a256(24 * 128 * f * 2) + _a256((1 + 2 * 32) * 4)
-    # pass schedule (also the default): chunks of whole shards within the hidden
-    # budget + the fp32 accumulator
+    # pass schedule (the default): chunks of whole shards within the hidden
+    # budget + the fp32 accumulator; the one-launch form holds two H chunk
+    # buffers and the dependency counters (2 chunks x 16 row pairs)
     ws = T.tsp_mlp_workspace_size(n, d, f, P, "swiglu", "bf16", "shard_passes")
-    assert ws == T.tsp_mlp_workspace_size(n, d, f, P, "swiglu", "bf16")
     acc = n * d * 4
+    assert ws == T.tsp_mlp_workspace_size(n, d, f, P, "swiglu", "bf16")
+    assert T.tsp_mlp_workspace_size(n, d, f, P, "swiglu", "bf16", "shard_passes_fused") == \
+        2 * (ws - acc) + acc + _a256((1 + 2 * 2 * 16) * 4)
     h = ws - acc
     assert h % (n * 2) == 0 and (h // (n * 2)) % (f // P) == 0
     assert h <= 64 << 20
