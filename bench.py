@@ -24,6 +24,8 @@ of the same workload (rank 0 only; other ranks exit at once).
 from __future__ import annotations
 
 import argparse
+import dataclasses
+import datetime
 import hashlib
 import json
 import os
@@ -41,7 +43,21 @@ sys.path.insert(0, ROOT)
 from workloads import WORKLOADS, LLAMA8B, make_inputs  # noqa: E402
 
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
-KERNEL_SOURCES = ["ptx.cuh", "pipeline.cuh", "pipeline2.cuh", "recipes.cuh", "fused.cuh", "fused2.cuh"]
+# the csrc headers each kernel is built from (a change to any of them voids its
+# committed ncu traffic figure)
+FORWARD_SOURCES = ["ptx.cuh", "pipeline.cuh", "pipeline2.cuh", "recipes.cuh"]
+
+
+def kernel_sources(kernel: str) -> list[str]:
+    if kernel.startswith("fused_fwd"):
+        return FORWARD_SOURCES + ["fused.cuh"]
+    if kernel.startswith("fused_passes"):
+        return FORWARD_SOURCES + ["fused.cuh", "fused2.cuh"]
+    if kernel.startswith(("bwd_", "wgrad_")):
+        return FORWARD_SOURCES + ["bwd_pair.cuh"]
+    if kernel.startswith("f32_"):
+        return ["simt_f32.cuh"]
+    return FORWARD_SOURCES
 
 
 def peaks():
@@ -55,9 +71,9 @@ def peaks():
             "source": "fallback"}
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(kernel: str) -> str:
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in kernel_sources(kernel):
         with open(os.path.join(ROOT, "sequence_transformer_mlp_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -71,7 +87,7 @@ def traffic_for(kernel: str, wl_name: str, launches_per_step: int):
     with open(PROFILE_TRAFFIC) as fh:
         j = json.load(fh)
     ent = j.get(wl_name, {}).get(kernel)
-    if not ent or ent.get("kernel_source_hash") != kernel_source_hash():
+    if not ent or ent.get("kernel_source_hash") != kernel_source_hash(kernel):
         return None
     return ent.get("dram_bytes_per_launch")
 
@@ -79,7 +95,7 @@ def traffic_for(kernel: str, wl_name: str, launches_per_step: int):
 class ClockSampler:
     """nvidia-smi sampled every 200 ms while running (SM clock and throttle reasons)."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -102,8 +118,18 @@ class ClockSampler:
                 stdout=self.out, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
-        time.sleep(0.3)
+        # wait for the first sample, so that sampling covers the timed region
+        t_end = time.time() + 5.0
+        while self.proc is not None and time.time() < t_end and os.path.getsize(self.path) == 0:
+            time.sleep(0.05)
+        self.t0 = self.t1 = None
         return self
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
 
     def __exit__(self, *exc):
         if self.proc is not None:
@@ -121,18 +147,28 @@ class ClockSampler:
         with open(self.path) as fh:
             for line in fh:
                 parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
+                if len(parts) >= 10:
+                    try:
+                        ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                    except ValueError:
+                        ts = None
+                    rows.append((ts, parts[1:]))
         os.unlink(self.path)
-        if not rows:
+        # only the samples taken while the timed region ran (all, if none fell in it)
+        window = [r for ts, r in rows
+                  if ts is not None and self.t0 is not None and self.t1 is not None
+                  and self.t0 <= ts <= self.t1]
+        use = window or [r for _, r in rows]
+        if not use:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        smax = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
-        loaded = [s for s in sm if s > 0.5 * smax] or sm
+        sm = [float(r[1]) for r in use if r[1].replace(".", "").isdigit()]
+        smax = max(float(r[2]) for r in use if r[2].replace(".", "").isdigit())
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
-        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax, "reasons": reasons,
-                "samples": len(rows)}
+        reasons = sorted({names[i] for r in use for i in range(4) if r[5 + i] == "Active"})
+        power = [float(r[3]) for r in use if r[3].replace(".", "").isdigit()]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": reasons, "samples": len(use), "samples_in_timed_region": len(window),
+                "power_w_median": statistics.median(power) if power else None}
 
 
 def reference_arm(args, wl, rank):
@@ -217,7 +253,7 @@ def end_to_end(args, inp, dev, step, Y, stream, barrier):
     inside the timed region.  Returns (ms per step, host X, host Y)."""
     n, d = inp["X"].shape
     Xh = inp["X"].pin_memory()
-    Yh = [torch.empty(n, d, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    Yh = [torch.empty(n, d, dtype=Y.dtype).pin_memory() for _ in range(2)]
     Xd = [torch.empty_like(dev["X"]) for _ in range(2)]
     Yd = [torch.empty_like(Y) for _ in range(2)]
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
@@ -259,7 +295,7 @@ def end_to_end(args, inp, dev, step, Y, stream, barrier):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=LLAMA8B.name, choices=sorted(WORKLOADS))
@@ -267,12 +303,19 @@ def main():
                     choices=["weight_shards", "tsp_ring", "shard_passes", "fused", "tsp_ring_fused",
                              "shard_passes_fused"],
                     help="override the workload's schedule")
+    ap.add_argument("--P", type=int, default=None,
+                    help="override the workload's number of logical weight shards")
     ap.add_argument("--ref-rows", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the host-buffer loop (used for short profiler runs)")
     args = ap.parse_args()
     wl = WORKLOADS[args.workload]
+    # traffic figures in the committed ncu summaries are for the workload's own P
+    traffic_key = wl.name
+    if args.P is not None and args.P != wl.P:
+        wl = dataclasses.replace(wl, P=args.P)
+        traffic_key = None
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -287,7 +330,6 @@ def main():
     torch.cuda.set_device(local)
     dist = None
     if world > 1:
-        import datetime
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
@@ -301,8 +343,10 @@ def main():
     n, d, f, P = wl.n, wl.d, wl.f, wl.P
     sched = args.sched or wl.sched
     stream = torch.cuda.current_stream()
-    Y = torch.empty(n, d, dtype=torch.bfloat16, device="cuda")
-    need = T.tsp_mlp_workspace_size(n, d, f, P, wl.act, "bf16", sched, backward=wl.backward)
+    dt = "f32" if wl.dtype == "f32" else "bf16"
+    tdt = torch.float32 if dt == "f32" else torch.bfloat16
+    Y = torch.empty(n, d, dtype=tdt, device="cuda")
+    need = T.tsp_mlp_workspace_size(n, d, f, P, wl.act, dt, sched, backward=wl.backward)
     ws = torch.empty(max(need, 1), dtype=torch.uint8, device="cuda")
     if wl.backward:
         dX = torch.empty(n, d, dtype=torch.bfloat16, device="cuda")
@@ -313,7 +357,7 @@ def main():
                            dtype=torch.uint8, device="cuda")
 
     def step(x=dev["X"], y=Y):
-        T.tsp_mlp_forward_ex(x, dev["A"], dev["Wu"], dev["B"], n, d, f, P, wl.act, "bf16", sched,
+        T.tsp_mlp_forward_ex(x, dev["A"], dev["Wu"], dev["B"], n, d, f, P, wl.act, dt, sched,
                              y, ws_f if wl.backward else ws,
                              ws_f.numel() if wl.backward else need, stream)
         if wl.backward:
@@ -333,11 +377,13 @@ def main():
     with ClockSampler(local) as clk:
         barrier()
         torch.cuda.synchronize()
+        clk.mark_start()
         e0.record(stream)
         for _ in range(args.steps):
             step()
         e1.record(stream)
         torch.cuda.synchronize()
+        clk.mark_end()
         barrier()
     T.tsp_trace_enable(False)
     ms = e0.elapsed_time(e1) / args.steps
@@ -357,6 +403,7 @@ def main():
     if dist is not None:
         ms, ms_e2e = max_over_ranks([ms, ms_e2e], dist, "cuda")
 
+    clocks = clk.summary()
     if rank == 0:
         pk = peaks()
         tflops = replica_throughput(world, flops, ms)
@@ -366,25 +413,32 @@ def main():
         launches_total = sum(v[0] for v in kstats.values())
         dom_flops_per_launch = kernel_flops_per_step(dom, wl) / (dom_launches / args.steps)
         achieved = dom_flops_per_launch / (dom_ms / dom_launches * 1e-3) / 1e12
-        traffic = traffic_for(dom, wl.name, dom_launches // args.steps)
+        traffic = traffic_for(dom, traffic_key, dom_launches // args.steps) if traffic_key else None
+        if dt == "f32":
+            # fp32 FMA on the CUDA cores: peak = SMs x 128 lanes x 2 FLOP x max SM clock
+            bound, peak, peak_src = "alu", fp32_alu_peak_tflops(clocks), "derived"
+        else:
+            bound, peak, peak_src = "tensor", pk["bf16_tflops"], pk["source"]
         line = {
             "metric": "sharded gated-MLP forward TFLOP/s" if not wl.backward
             else "sharded gated-MLP forward+backward TFLOP/s",
             "value": tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic (seeded torch.randn, cast to bf16)",
+            "scaling": "weak", "vs_baseline": None, "dtype": dt,
+            "data": f"synthetic (seeded torch.randn, cast to {dt})",
             "tokens_per_s": world * n / (ms * 1e-3),
             "pct_of_bf16_peak": 100.0 * tflops / (world * pk["bf16_tflops"]),
             "pct_of_bf16_peak_sustained": 100.0 * tflops / (world * pk["bf16_tflops_sustained"]),
             "config": {"workload": wl.name, "n_tokens": n, "d_model": d, "d_ff": f, "P": P,
                        "act": wl.act, "schedule": sched, "parallelism": f"replicas{world}",
-                       "l2": "inputs larger than L2 (weights 3 x d x f bf16), no flush"},
-            "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved,
-                         "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                         "frac": achieved / pk["bf16_tflops"],
-                         "frac_of_sustained": achieved / pk["bf16_tflops_sustained"],
-                         "peak_source": pk["source"], "traffic": traffic,
+                       "l2": "inputs larger than L2 (weights 3 x d x f bf16), no flush"
+                       if dt == "bf16" else "inputs fit in L2 (launch-latency bound), no flush"},
+            "roofline": {"bound": bound, "kernel": dom, "achieved": achieved,
+                         "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak,
+                         "frac_of_sustained": achieved / pk["bf16_tflops_sustained"]
+                         if dt == "bf16" else None,
+                         "peak_source": peak_src, "traffic": traffic,
                          "flops_per_launch": dom_flops_per_launch,
                          "share_of_kernel_time": dom_ms / total_k if total_k else None},
             "kernels": {k: {"launches": v[0], "ms_per_launch": v[1] / v[0]}
@@ -395,7 +449,7 @@ def main():
                 "h2d_bytes_per_step": Xh.numel() * Xh.element_size(),
                 "d2h_bytes_per_step": Yh.numel() * Yh.element_size(),
                 "ms_per_step": ms_e2e},
-            "clocks": clk.summary(),
+            "clocks": clocks,
         }
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(wl)
@@ -404,6 +458,13 @@ def main():
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def fp32_alu_peak_tflops(clocks: dict) -> float:
+    """fp32 FMA peak of the device: SMs x 128 fp32 lanes x 2 FLOP x max SM clock."""
+    props = torch.cuda.get_device_properties(torch.cuda.current_device())
+    mhz = clocks.get("sm_max_mhz") or 1965.0
+    return props.multi_processor_count * 128 * 2 * mhz * 1e6 / 1e12
 
 
 def kernel_flops_per_step(kernel: str, wl) -> float:
@@ -431,6 +492,9 @@ def kernel_flops_per_step(kernel: str, wl) -> float:
         "wgrad_gelu_a": 2 * n * d * f,
         "dgrad_accum_swiglu": 2 * 2 * n * d * f,
         "dgrad_accum_gelu": 2 * n * d * f,
+        "f32_hidden_swiglu": 2 * 2 * n * d * f,
+        "f32_hidden_gelu": 2 * n * d * f,
+        "f32_down": 2 * n * d * f,
     }[kernel]
 
 

@@ -92,9 +92,12 @@ typedef enum {
      * adds its partial output into the shard's fp32 accumulator in place.
      * Needs n % P == 0. */
     TSP_SCHED_TSP_RING = 1,
-    /* Weight-shard schedule as separate passes: per chunk of shards one
-     * gate/up launch and one down-projection launch whose partial output is
-     * added into an fp32 [n][d_model] accumulator in place. */
+    /* Weight-shard schedule as separate passes: per chunk of whole shards
+     * (as many as fit a 512 MB hidden buffer) one gate/up launch and one
+     * down-projection launch.  With several chunks each partial output is
+     * added into an fp32 [n][d_model] accumulator in place; with one chunk
+     * the down projection's tensor-memory accumulator sums the shards in
+     * order and writes Y directly. */
     TSP_SCHED_SHARD_PASSES = 2,
     /* Weight-shard schedule as one persistent launch (bf16): per block of 128
      * tokens the hidden activations go to a ring of row-block slots and the

@@ -1,0 +1,309 @@
+// bwd_pair.cuh -- the backward's paired recipes for the pipeline of
+// pipeline2.cuh: the weight gradients (WgradPair) and the hidden layer's
+// backward as two GEMMs (BwdGateUpPair, DhPair).  The input gradient reuses
+// DownAccumPair with K-major weights.
+#pragma once
+
+#include "pipeline2.cuh"
+
+namespace tspmlp {
+
+// ============================================================================
+// Paired weight gradients (see Wgrad): both operands MN-major, K = tokens.
+// Tile = 256 output rows x NCOLS output columns; CTA r stages 128 of the rows
+// (A) and NCOLS/2 of the columns (B).  SPLIT: CTA 0 stages dG, CTA 1 dU, so
+// TMEM columns 0-127 hold dW_gate and 128-255 dW_up.
+template <int NCOLS, bool SPLIT>
+struct WgradPair {
+    using Base = Wgrad<NCOLS, SPLIT>;
+    using Params = typename Base::Params;
+    static constexpr const char* kName = Base::kName;
+    static constexpr int kBK = 64;
+    static constexpr int kABytes = 128 * kBK * 2;
+    static constexpr int kStageBytes = kABytes + (NCOLS / 2) * kBK * 2;
+    static constexpr int kStages = kStageBytes <= 24576 ? 8 : 6;
+    static constexpr int kAccCols = 256, kAccBufs = 2;
+    static constexpr int kTileCols = Base::kTileCols;
+    static constexpr uint32_t kIdesc = make_idesc_bf16(256, NCOLS, true, true);
+    struct Tile {
+        int mi, nj;
+    };
+    __host__ __device__ static int num_tiles(const Params& p) {
+        return ((p.m_valid + 255) / 256) * ((p.n_valid + kTileCols - 1) / kTileCols);
+    }
+    // Both operands span all K = tokens, so a wave of concurrent tiles re-reads
+    // every block of the operand whose index varies fastest.  That index runs
+    // over the operand with fewer blocks (X or dY: n x d_model, which L2
+    // holds), so the larger one (H, dG/dU: n x d_ff) streams from HBM once.
+    __device__ static Tile tile(const Params& p, int t) {
+        const int mt = (p.m_valid + 255) / 256;
+        const int nt = (p.n_valid + kTileCols - 1) / kTileCols;
+        if (mt <= nt) return Tile{t % mt, t / mt};
+        return Tile{t / nt, t % nt};
+    }
+    __device__ static int num_kb(const Params& p, const Tile&) { return (p.ntok + kBK - 1) / kBK; }
+    __device__ static void prefetch(const Params& p) { Base::prefetch(p); }
+    __device__ static void load(const Params& p, const Tile& ti, int kb, uint32_t rank, uint32_t st,
+                                uint32_t bar) {
+        const int k0 = kb * kBK;
+        const int a = p.a_col0 + ti.mi * 256 + static_cast<int>(rank) * 128;
+        tma_load_2d_pair(st, &p.tmA, bar, a, k0);
+        tma_load_2d_pair(st + 8192, &p.tmA, bar, a + 64, k0);
+        const uint32_t b = st + kABytes;
+        if (SPLIT) {
+            const int c = p.b_col0 + ti.nj * kTileCols;
+            const CUtensorMap* src = rank == 0 ? &p.tmB0 : &p.tmB1;
+#pragma unroll
+            for (int i = 0; i < NCOLS / 128; ++i) tma_load_2d_pair(b + 8192 * i, src, bar, c + 64 * i, k0);
+        } else {
+            const int c = p.b_col0 + ti.nj * NCOLS + static_cast<int>(rank) * (NCOLS / 2);
+#pragma unroll
+            for (int i = 0; i < NCOLS / 128; ++i) tma_load_2d_pair(b + 8192 * i, &p.tmB0, bar, c + 64 * i, k0);
+        }
+    }
+    __device__ static void mma(const Tile&, int kb, uint32_t st, uint32_t acc) {
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t a = make_smem_desc(st + 2048 * kk, 8192, 1024, kLayoutSW128);
+            const uint64_t b = make_smem_desc(st + kABytes + 2048 * kk, 8192, 1024, kLayoutSW128);
+            umma_bf16_pair(acc, a, b, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+        }
+    }
+    __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t rank, uint32_t acc,
+                                    int q, int lane) {
+        typename Base::Tile t1{2 * ti.mi + static_cast<int>(rank), ti.nj};
+        Base::epilogue(p, t1, acc, q, lane);
+    }
+};
+
+// ============================================================================
+// Backward of the hidden layer as two double-buffered paired GEMMs.
+//
+// BwdGateUpPair: the recomputed gate/up projection (as FwdHiddenPair, K =
+// d_model) whose epilogue writes, per hidden unit,
+//   SwiGLU: H = SiLU(G) U (bf16), S1 = SiLU(G), S2 = U SiLU'(G)   (fp32)
+//   GeLU:   H = GeLU(G) (bf16),  S1 = GeLU'(G)                     (fp32)
+// DhPair: dH = dY . W_down[c..]^T (K = d_model, both operands K-major) whose
+// epilogue forms the pre-activation gradients from the stored factors,
+//   SwiGLU: dU = dH S1, dG = dH S2;   GeLU: dG = dH S1          (bf16)
+// -- the derivatives of the forward definition, as in BwdHidden; the factors
+// stay fp32 so the only rounding is that of dG / dU, as there.
+struct BwdGateUpParams {
+    CUtensorMap tmX;  // X [n][d], box {64, 128}
+    CUtensorMap tmG;  // W_gate / A [d][f], box {64, 64}
+    CUtensorMap tmU;  // W_up [d][f], box {64, 64} (SwiGLU)
+    int n, d, col_base, width;
+    __nv_bfloat16* H;  // [n][width]
+    float* S1;         // [n][width]
+    float* S2;         // [n][width] (SwiGLU)
+    long long ld;
+};
+
+template <int ACT>
+struct BwdGateUpPair {
+    using Params = BwdGateUpParams;
+    static constexpr const char* kName = ACT == 1 ? "bwd_gate_up_swiglu" : "bwd_gate_up_gelu";
+    static constexpr int kBK = 64;
+    static constexpr int kOut = ACT == 1 ? 128 : 256;
+    static constexpr int kABytes = 128 * kBK * 2;
+    static constexpr int kStageBytes = kABytes + 128 * kBK * 2;
+    static constexpr int kStages = 6;
+    static constexpr int kAccCols = 256, kAccBufs = 2;
+    static constexpr uint32_t kIdesc = make_idesc_bf16(256, 256, false, true);
+    struct Tile {
+        int mi, nj;
+    };
+    __host__ __device__ static int num_tiles(const Params& p) {
+        return ((p.n + 255) / 256) * ((p.width + kOut - 1) / kOut);
+    }
+    __device__ static Tile tile(const Params& p, int t) {
+        const int mt = (p.n + 255) / 256;
+        return Tile{t % mt, t / mt};
+    }
+    __device__ static int num_kb(const Params& p, const Tile&) { return (p.d + kBK - 1) / kBK; }
+    __device__ static void prefetch(const Params& p) {
+        tma_prefetch_desc(&p.tmX);
+        tma_prefetch_desc(&p.tmG);
+        if (ACT == 1) tma_prefetch_desc(&p.tmU);
+    }
+    __device__ static void load(const Params& p, const Tile& ti, int kb, uint32_t rank, uint32_t st,
+                                uint32_t bar) {
+        const int k0 = kb * kBK;
+        tma_load_2d_pair(st, &p.tmX, bar, k0, ti.mi * 256 + static_cast<int>(rank) * 128);
+        const int c = p.col_base + ti.nj * kOut;
+        if (ACT == 1) {
+            const CUtensorMap* w = rank == 0 ? &p.tmG : &p.tmU;
+            tma_load_2d_pair(st + kABytes, w, bar, c, k0);
+            tma_load_2d_pair(st + kABytes + 8192, w, bar, c + 64, k0);
+        } else {
+            const int cr = c + static_cast<int>(rank) * 128;
+            tma_load_2d_pair(st + kABytes, &p.tmG, bar, cr, k0);
+            tma_load_2d_pair(st + kABytes + 8192, &p.tmG, bar, cr + 64, k0);
+        }
+    }
+    __device__ static void mma(const Tile&, int kb, uint32_t st, uint32_t acc) {
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t a = make_smem_desc(st + 32 * kk, 16, 1024, kLayoutSW128);
+            const uint64_t b = make_smem_desc(st + kABytes + 2048 * kk, 8192, 1024, kLayoutSW128);
+            umma_bf16_pair(acc, a, b, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+        }
+    }
+    __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t rank, uint32_t acc,
+                                    int q, int lane) {
+        const int row = ti.mi * 256 + static_cast<int>(rank) * 128 + q * 32 + lane;
+        const bool row_ok = row < p.n;
+        const long long off = static_cast<long long>(row) * p.ld;
+        const uint32_t t0 = acc + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll 1
+        for (int cc = 0; cc < (ACT == 1 ? 4 : 8); ++cc) {
+            uint32_t g[32], pk[16], s1[32], s2[32];
+            tmem_ld_32x32b_x32(t0 + 32 * cc, g);
+            if (ACT == 1) {
+                uint32_t u[32];
+                tmem_ld_32x32b_x32(t0 + 128 + 32 * cc, u);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float gv = __uint_as_float(g[i]), uv = __uint_as_float(u[i]);
+                    const float sg = 1.0f / (1.0f + __expf(-gv));
+                    const float si = gv * sg;
+                    s1[i] = __float_as_uint(si);
+                    s2[i] = __float_as_uint(uv * sg * (1.0f + gv * (1.0f - sg)));
+                    g[i] = __float_as_uint(si * uv);
+                }
+            } else {
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float z = __uint_as_float(g[i]);
+                    const float cdf = 0.5f * (1.0f + erff(z * 0.70710678118654752440f));
+                    const float pdf = 0.39894228040143267794f * __expf(-0.5f * z * z);
+                    s1[i] = __float_as_uint(cdf + z * pdf);
+                    g[i] = __float_as_uint(z * cdf);
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                pk[i] = pack_bf16x2(__uint_as_float(g[2 * i]), __uint_as_float(g[2 * i + 1]));
+            const int c0 = ti.nj * kOut + 32 * cc;
+            if (row_ok) {
+                store_bf16x32(p.H + off + c0, pk, p.width - c0);
+                store_f32x32(p.S1 + off + c0, s1, p.width - c0);
+                if (ACT == 1) store_f32x32(p.S2 + off + c0, s2, p.width - c0);
+            }
+        }
+    }
+};
+
+struct DhParams {
+    CUtensorMap tmDY;  // dY [n][d], box {64, 128}
+    CUtensorMap tmD;   // W_down / B [f][d], box {64, 128} (K-major: rows are hidden units)
+    int n, d, col_base, width;
+    const float* S1;   // [n][width]
+    const float* S2;   // [n][width] (SwiGLU)
+    __nv_bfloat16* dG; // [n][width]
+    __nv_bfloat16* dU; // [n][width] (SwiGLU)
+    long long ld;
+};
+
+template <int ACT>
+struct DhPair {
+    using Params = DhParams;
+    static constexpr const char* kName = ACT == 1 ? "bwd_dh_swiglu" : "bwd_dh_gelu";
+    static constexpr int kBK = 64;
+    static constexpr int kABytes = 128 * kBK * 2;
+    static constexpr int kStageBytes = kABytes + 128 * kBK * 2;
+    static constexpr int kStages = 6;
+    static constexpr int kAccCols = 256, kAccBufs = 2;
+    static constexpr uint32_t kIdesc = make_idesc_bf16(256, 256, false, false);
+    struct Tile {
+        int mi, nj;
+    };
+    __host__ __device__ static int num_tiles(const Params& p) {
+        return ((p.n + 255) / 256) * ((p.width + 255) / 256);
+    }
+    __device__ static Tile tile(const Params& p, int t) {
+        const int mt = (p.n + 255) / 256;
+        return Tile{t % mt, t / mt};
+    }
+    __device__ static int num_kb(const Params& p, const Tile&) { return (p.d + kBK - 1) / kBK; }
+    __device__ static void prefetch(const Params& p) {
+        tma_prefetch_desc(&p.tmDY);
+        tma_prefetch_desc(&p.tmD);
+    }
+    __device__ static void load(const Params& p, const Tile& ti, int kb, uint32_t rank, uint32_t st,
+                                uint32_t bar) {
+        const int k0 = kb * kBK;
+        tma_load_2d_pair(st, &p.tmDY, bar, k0, ti.mi * 256 + static_cast<int>(rank) * 128);
+        tma_load_2d_pair(st + kABytes, &p.tmD, bar, k0,
+                         p.col_base + ti.nj * 256 + static_cast<int>(rank) * 128);
+    }
+    __device__ static void mma(const Tile&, int kb, uint32_t st, uint32_t acc) {
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t a = make_smem_desc(st + 32 * kk, 16, 1024, kLayoutSW128);
+            const uint64_t b = make_smem_desc(st + kABytes + 32 * kk, 16, 1024, kLayoutSW128);
+            umma_bf16_pair(acc, a, b, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+        }
+    }
+    __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t rank, uint32_t acc,
+                                    int q, int lane) {
+        const int row = ti.mi * 256 + static_cast<int>(rank) * 128 + q * 32 + lane;
+        const bool row_ok = row < p.n;
+        const long long off = static_cast<long long>(row) * p.ld;
+        const uint32_t t0 = acc + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll 1
+        for (int cc = 0; cc < 8; ++cc) {
+            uint32_t dh[32], pg[16], pu[16];
+            tmem_ld_32x32b_x32(t0 + 32 * cc, dh);
+            tmem_ld_wait();
+            const int c0 = ti.nj * 256 + 32 * cc;
+            const int valid = p.width - c0;
+            if (!row_ok || valid <= 0) continue;
+            float f1[32], f2[32];
+            if (valid >= 32) {
+                const float4* a4 = reinterpret_cast<const float4*>(p.S1 + off + c0);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float4 v = a4[i];
+                    f1[4 * i] = v.x;
+                    f1[4 * i + 1] = v.y;
+                    f1[4 * i + 2] = v.z;
+                    f1[4 * i + 3] = v.w;
+                }
+                if (ACT == 1) {
+                    const float4* b4 = reinterpret_cast<const float4*>(p.S2 + off + c0);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float4 v = b4[i];
+                        f2[4 * i] = v.x;
+                        f2[4 * i + 1] = v.y;
+                        f2[4 * i + 2] = v.z;
+                        f2[4 * i + 3] = v.w;
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    f1[i] = i < valid ? p.S1[off + c0 + i] : 0.f;
+                    f2[i] = (ACT == 1 && i < valid) ? p.S2[off + c0 + i] : 0.f;
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float a0 = __uint_as_float(dh[2 * i]), a1 = __uint_as_float(dh[2 * i + 1]);
+                if (ACT == 1) {
+                    pu[i] = pack_bf16x2(a0 * f1[2 * i], a1 * f1[2 * i + 1]);
+                    pg[i] = pack_bf16x2(a0 * f2[2 * i], a1 * f2[2 * i + 1]);
+                } else {
+                    pg[i] = pack_bf16x2(a0 * f1[2 * i], a1 * f1[2 * i + 1]);
+                }
+            }
+            store_bf16x32(p.dG + off + c0, pg, valid);
+            if (ACT == 1) store_bf16x32(p.dU + off + c0, pu, valid);
+        }
+    }
+};
+
+}  // namespace tspmlp

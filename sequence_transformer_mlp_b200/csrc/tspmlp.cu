@@ -19,6 +19,7 @@
 #include <vector>
 
 #include "../../include/tspmlp.h"
+#include "bwd_pair.cuh"
 #include "fused.cuh"
 #include "fused2.cuh"
 #include "pipeline2.cuh"
@@ -30,9 +31,15 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
-// Scratch budgets: the hidden chunk(s) of one pass should stay resident in the
-// 126 MB L2 between the producing and the consuming kernel.
-constexpr size_t kFwdHiddenBudget = 64ull << 20;   // one bf16 [rows][C] buffer
+// Scratch budgets.  The pass schedule's hidden buffer holds as many whole
+// shards as fit in kFwdHiddenBudget: every extra chunk costs a read-modify-
+// write pass of the fp32 [n][d_model] accumulator, which measured dearer than
+// keeping the chunk's H resident in the 126 MB L2 (one 117 MB chunk beat two
+// 59 MB chunks on the Llama-3-8B shape, and the 70B shape gained ~5% going
+// from eight chunks to one or two).  The fused schedules keep their H ring
+// (or two H chunk buffers) within L2-sized budgets: their consumers read H
+// while it is being produced.
+constexpr size_t kFwdHiddenBudget = 512ull << 20;  // one bf16 [rows][C] buffer
 constexpr size_t kFusedRingBudget = 96ull << 20;   // the fused schedule's H ring
 constexpr size_t kFusedPassesBudget = 128ull << 20; // two H chunk buffers of the one-launch passes
 // H, dG, dU (bf16) and the fp32 activation-derivative factors together.  The
@@ -109,7 +116,6 @@ bool tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
 }
 
 constexpr CUtensorMapSwizzle SW128 = CU_TENSOR_MAP_SWIZZLE_128B;
-constexpr CUtensorMapSwizzle SW64 = CU_TENSOR_MAP_SWIZZLE_64B;
 
 // ---------------------------------------------------------------------------
 // tracing: CUDA events around each launch, on the launching stream
@@ -468,7 +474,9 @@ FwdPlan plan_forward_budget(int64_t n, int64_t d, int64_t f, int P, tsp_dtype_t 
             pl.sync_bytes = static_cast<size_t>(1 + 2 * pl.chunks.size() * ((n + 255) / 256)) * 4;
         }
     } else {
-        for (int w = 0; w < P; ++w) pl.chunks.push_back({w * fs, fs});
+        // fp32: chunks of whole shards within the same budget (no sub-shard cuts)
+        const int64_t mc = max_chunk_cols(budget, static_cast<size_t>(n) * 4);
+        pl.chunks = plan_chunks(f, P, std::max(mc, fs));
     }
     int64_t wmax = 0;
     for (auto& c : pl.chunks) wmax = std::max(wmax, c.width);
@@ -768,33 +776,55 @@ tsp_status_t forward_bf16(const void* X, const void* Wg, const void* Wu, const v
     return TSP_OK;
 }
 
+// Grid of TM x TM output tiles over rows x cols for each segment.
+template <int TM>
+dim3 f32_grid(int64_t cols, int rows, int segs) {
+    return dim3(static_cast<unsigned>((cols + TM - 1) / TM), static_cast<unsigned>((rows + TM - 1) / TM),
+                static_cast<unsigned>(segs));
+}
+
+// Large tiles when they make at least one block per SM, small ones otherwise.
+bool f32_small_tiles(int64_t cols, int rows, int segs, int sms) {
+    const dim3 g = f32_grid<kF32TileLarge>(cols, rows, segs);
+    return static_cast<int64_t>(g.x) * g.y * g.z < sms;
+}
+
+template <int ACT>
+void launch_f32_hidden(const float* X, const float* Wg, const float* Wu, int64_t d, int64_t f,
+                       const SegGeom& g, int64_t width, float* H, cudaStream_t st, int sms) {
+    if (f32_small_tiles(width, g.seg_rows, g.num_segs, sms))
+        f32_hidden_kernel<ACT, kF32TileSmall, kF32KSmall>
+            <<<f32_grid<kF32TileSmall>(width, g.seg_rows, g.num_segs), 256, 0, st>>>(
+                X, Wg, Wu, static_cast<int>(d), static_cast<int>(f), g, static_cast<int>(width), H, width);
+    else
+        f32_hidden_kernel<ACT, kF32TileLarge, kF32KLarge>
+            <<<f32_grid<kF32TileLarge>(width, g.seg_rows, g.num_segs), 256, 0, st>>>(
+                X, Wg, Wu, static_cast<int>(d), static_cast<int>(f), g, static_cast<int>(width), H, width);
+}
+
 tsp_status_t forward_f32(const float* X, const float* Wg, const float* Wu, const float* Wd,
                          int64_t n, int64_t d, int64_t f, int P, tsp_act_t act, const FwdPlan& pl,
-                         float* Y, void* ws, cudaStream_t st) {
+                         float* Y, void* ws, cudaStream_t st, int sms) {
     float* H = static_cast<float*>(ws);
     const int64_t fs = f / P;
     auto run = [&](const SegGeom& g, int64_t width, int first) -> tsp_status_t {
-        dim3 gh(static_cast<unsigned>((width + kF32Tile - 1) / kF32Tile),
-                static_cast<unsigned>((g.seg_rows + kF32Tile - 1) / kF32Tile),
-                static_cast<unsigned>(g.num_segs));
         TraceRec rec;
         bool traced = trace_begin(st, &rec, act == TSP_ACT_SWIGLU ? "f32_hidden_swiglu" : "f32_hidden_gelu");
         if (act == TSP_ACT_SWIGLU)
-            f32_hidden_kernel<1><<<gh, 256, 0, st>>>(X, Wg, Wu, static_cast<int>(d),
-                                                     static_cast<int>(f), g, static_cast<int>(width),
-                                                     H, width);
+            launch_f32_hidden<1>(X, Wg, Wu, d, f, g, width, H, st, sms);
         else
-            f32_hidden_kernel<0><<<gh, 256, 0, st>>>(X, Wg, Wu, static_cast<int>(d),
-                                                     static_cast<int>(f), g, static_cast<int>(width),
-                                                     H, width);
+            launch_f32_hidden<0>(X, Wg, Wu, d, f, g, width, H, st, sms);
         if (traced) trace_end(st, &rec);
         if (cudaGetLastError() != cudaSuccess) return TSP_ERR_CUDA;
-        dim3 gd(static_cast<unsigned>((d + kF32Tile - 1) / kF32Tile),
-                static_cast<unsigned>((g.seg_rows + kF32Tile - 1) / kF32Tile),
-                static_cast<unsigned>(g.num_segs));
         traced = trace_begin(st, &rec, "f32_down");
-        f32_down_kernel<<<gd, 256, 0, st>>>(H, width, Wd, static_cast<int>(d), g,
-                                            static_cast<int>(width), first, Y);
+        if (f32_small_tiles(d, g.seg_rows, g.num_segs, sms))
+            f32_down_kernel<kF32TileSmall, kF32KSmall>
+                <<<f32_grid<kF32TileSmall>(d, g.seg_rows, g.num_segs), 256, 0, st>>>(
+                    H, width, Wd, static_cast<int>(d), g, static_cast<int>(width), first, Y);
+        else
+            f32_down_kernel<kF32TileLarge, kF32KLarge>
+                <<<f32_grid<kF32TileLarge>(d, g.seg_rows, g.num_segs), 256, 0, st>>>(
+                    H, width, Wd, static_cast<int>(d), g, static_cast<int>(width), first, Y);
         if (traced) trace_end(st, &rec);
         return cudaGetLastError() == cudaSuccess ? TSP_OK : TSP_ERR_CUDA;
     };
@@ -1074,7 +1104,7 @@ tsp_status_t tsp_mlp_forward_ex(const void* X, const void* Wg, const void* Wu, c
     if (dt == TSP_DT_F32)
         return forward_f32(static_cast<const float*>(X), static_cast<const float*>(Wg),
                            static_cast<const float*>(Wu), static_cast<const float*>(Wd), n, d, f, P,
-                           act, pl, static_cast<float*>(Y), ws, st);
+                           act, pl, static_cast<float*>(Y), ws, st, di.sms);
     if (act == TSP_ACT_SWIGLU)
         return forward_bf16<1>(X, Wg, Wu, Wd, n, d, f, P, pl, Y, ws, st, dev, di.sms);
     return forward_bf16<0>(X, Wg, Wu, Wd, n, d, f, P, pl, Y, ws, st, dev, di.sms);

@@ -52,8 +52,11 @@ def _a256(b):
 
 
 def test_workspace_sizes_follow_the_schedule(lib):
-    # fp32 weight-shard schedule: one shard's hidden block, Y accumulates in place
-    assert T.tsp_mlp_workspace_size(64, 128, 512, 2, "gelu", "f32") == 64 * 256 * 4
+    # fp32 weight-shard schedule: the hidden block of every shard in one chunk
+    # (Y accumulates in place only when there are several chunks)
+    assert T.tsp_mlp_workspace_size(64, 128, 512, 2, "gelu", "f32") == 64 * 512 * 4
+    # fp32 TSP ring: one ring step's hidden block for all sequence shards
+    assert T.tsp_mlp_workspace_size(64, 128, 512, 2, "gelu", "f32", "tsp_ring") == 64 * 256 * 4
     # bf16 fused schedule: an H ring of row-block slots (128 x d_ff) and the
     # per-row-block counters; 2 row blocks -> 2 slots
     assert T.tsp_mlp_workspace_size(256, 64, 512, 1, "swiglu", "bf16", "fused") == \
@@ -62,17 +65,21 @@ def test_workspace_sizes_follow_the_schedule(lib):
     n, d, f, P = 4096, 4096, 14336, 8
     assert T.tsp_mlp_workspace_size(n, d, f, P, "swiglu", "bf16", "fused") == \
         _a256(24 * 128 * f * 2) + _a256((1 + 2 * 32) * 4)
-    # pass schedule (the default): chunks of whole shards within the hidden
-    # budget + the fp32 accumulator; the one-launch form holds two H chunk
-    # buffers and the dependency counters (2 chunks x 16 row pairs)
+    # pass schedule (the default): chunks of whole shards within the 512 MB
+    # hidden budget -- here all eight shards in one chunk, so no fp32
+    # accumulator; the one-launch form holds two H chunk buffers within 128 MB
+    # (2 chunks of 4 shards), the accumulator and the dependency counters
+    # (2 chunks x 16 row pairs)
     ws = T.tsp_mlp_workspace_size(n, d, f, P, "swiglu", "bf16", "shard_passes")
     acc = n * d * 4
-    assert ws == T.tsp_mlp_workspace_size(n, d, f, P, "swiglu", "bf16")
+    assert ws == T.tsp_mlp_workspace_size(n, d, f, P, "swiglu", "bf16") == n * f * 2
     assert T.tsp_mlp_workspace_size(n, d, f, P, "swiglu", "bf16", "shard_passes_fused") == \
-        2 * (ws - acc) + acc + _a256((1 + 2 * 2 * 16) * 4)
-    h = ws - acc
-    assert h % (n * 2) == 0 and (h // (n * 2)) % (f // P) == 0
-    assert h <= 64 << 20
+        2 * (n * f // 2 * 2) + acc + _a256((1 + 2 * 2 * 16) * 4)
+    # 70B shape: 470 MB of H in one chunk; 32768 tokens of the 8B shape: 940 MB
+    # of H in two chunks of four shards + the accumulator
+    assert T.tsp_mlp_workspace_size(8192, 8192, 28672, 8, "swiglu", "bf16") == 8192 * 28672 * 2
+    assert T.tsp_mlp_workspace_size(32768, d, f, P, "swiglu", "bf16") == \
+        32768 * (f // 2) * 2 + 32768 * d * 4
     # single chunk: no accumulator
     assert T.tsp_mlp_workspace_size(256, 64, 512, 1, "swiglu", "bf16", "shard_passes") == \
         256 * 512 * 2

@@ -31,6 +31,7 @@ def check(got, ref, what):
     mx = float(np.abs(ref).max())
     err = float(np.abs(got - ref).max())
     fro = float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300))
+    print(f"PARITY {what} max_rel={err / mx:.3e} fro={fro:.3e}")  # shown with pytest -s
     assert err <= 1e-2 * mx, f"{what}: max|d|/max|ref| = {err / mx:.3e}"
     assert fro <= 5e-3, f"{what}: rel Frobenius {fro:.3e}"
 

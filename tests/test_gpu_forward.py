@@ -29,6 +29,7 @@ def check(got, ref, dtype, what=""):
     mx = float(np.abs(ref).max())
     err = float(np.abs(got - ref).max())
     fro = float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300))
+    print(f"PARITY {what} max_rel={err / mx:.3e} fro={fro:.3e}")  # shown with pytest -s
     if dtype == "f32":
         assert err <= 1e-5 * mx and fro <= 1e-5, f"{what}: max {err / mx:.3e} fro {fro:.3e}"
     else:
@@ -75,6 +76,17 @@ def test_gelu_fp32_any_P_and_schedule(P, sched):
     Y = gpu_forward(inp, P, "gelu", sched)
     ref = oracle.mlp_forward(inp["X"], inp["A"], None, inp["B"], "gelu")
     check(Y, ref, "f32", f"P={P} {sched}")
+
+
+@pytest.mark.parametrize("act", ["gelu", "swiglu"])
+def test_fp32_large_tiles(act):
+    """Enough hidden tiles for the 64 x 64 fp32 tiles (the down projection,
+    with fewer, takes the 16 x 16 ones); ragged in every dimension."""
+    wl = small(act, "f32", 700, 96, 3 * 600, 3, seed=6, w_std=0.1)
+    inp = make_inputs(wl)
+    Y = gpu_forward(inp, wl.P, act)
+    ref = oracle.mlp_forward(inp["X"], inp["A"], inp["Wu"], inp["B"], act)
+    check(Y, ref, "f32", wl.name)
 
 
 @pytest.mark.parametrize("act", ["gelu", "swiglu"])
@@ -217,16 +229,17 @@ def _full_inputs(wl):
     return inp, {k: to_dev(v) for k, v in inp.items()}
 
 
-def _sampled_check(wl, inp, Y_dev, rows, act="swiglu", sched="weight_shards"):
+def _sampled_check(wl, inp, Y_dev, rows, act="swiglu", sched="weight_shards", P=None):
+    P = wl.P if P is None else P
     Y = Y_dev[rows].float().cpu().double().numpy()
     X = inp["X"][rows]
-    if sched == "tsp_ring":
+    if sched.startswith("tsp_ring"):
         # the ring result of a row is its sequence shard's ring-ordered sum;
         # within fp64 it equals the unsharded block (pinned in the oracle tests)
         ref = oracle.mlp_forward(X, inp["A"], inp["Wu"], inp["B"], act)
     else:
-        ref = oracle.mlp_sharded(X, inp["A"], inp["Wu"], inp["B"], act, wl.P)
-    return check(Y, ref, "bf16", wl.name)
+        ref = oracle.mlp_sharded(X, inp["A"], inp["Wu"], inp["B"], act, P)
+    return check(Y, ref, "bf16", f"{wl.name} P={P} {sched}")
 
 
 @pytest.fixture(scope="module")
@@ -242,7 +255,7 @@ def test_llama8b_shape_sampled_rows(llama8b, P, sched):
     Y = T.mlp_forward(dev["X"], dev["A"], dev["Wu"], dev["B"], P, "swiglu", sched=sched)
     assert T.tsp_poll_device_error() == T.TSP_OK
     rows = sample_rows(LLAMA8B.n, 24, LLAMA8B.seed)
-    _sampled_check(LLAMA8B, inp, Y, rows)
+    _sampled_check(LLAMA8B, inp, Y, rows, sched=sched, P=P)
 
 
 @pytest.mark.parametrize("sched", ["tsp_ring", "tsp_ring_fused"])
@@ -255,7 +268,7 @@ def test_tsp_ring_long_context_sampled_rows(sched):
     ns = TSP_RING.n // TSP_RING.P
     rows = sorted(set(sample_rows(TSP_RING.n, 16, TSP_RING.seed) +
                       [s * ns for s in range(TSP_RING.P)] + [s * ns + ns - 1 for s in range(TSP_RING.P)]))
-    _sampled_check(TSP_RING, inp, Y, rows, sched="tsp_ring")
+    _sampled_check(TSP_RING, inp, Y, rows, sched=sched)
 
 
 def test_llama70b_shape_sampled_rows():
