@@ -88,9 +88,14 @@ typedef enum {
      * fastest measured implementation: TSP_SCHED_SHARD_PASSES for bf16). */
     TSP_SCHED_WEIGHT_SHARDS = 0,
     /* Folded tensor-and-sequence ring: tokens form P equal sequence shards;
-     * at ring step t sequence shard s meets weight shard (s + t) mod P and
-     * adds its partial output into the shard's fp32 accumulator in place.
-     * Needs n % P == 0. */
+     * at ring step t sequence shard s meets weight shard (s + t) mod P, and
+     * each sequence shard sums its partial outputs in that ring order.  Needs
+     * n % P == 0.  bf16 with (d_ff / P) % 64 == 0: per group of sequence
+     * shards (as many as fit 512 MB of hidden activations) one gate/up launch
+     * over all d_ff columns and one down projection whose K loop runs over
+     * the weight shards in each sequence shard's ring order, summing in
+     * tensor memory.  Otherwise: per ring step one gate/up and one down
+     * launch, the partial outputs added into an fp32 accumulator in place. */
     TSP_SCHED_TSP_RING = 1,
     /* Weight-shard schedule as separate passes: per chunk of whole shards
      * (as many as fit a 512 MB hidden buffer) one gate/up launch and one

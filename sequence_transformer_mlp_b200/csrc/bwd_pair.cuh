@@ -79,23 +79,89 @@ struct WgradPair {
 // ============================================================================
 // Backward of the hidden layer as two double-buffered paired GEMMs.
 //
+// DhPair: dH = dY . W_down[c..]^T (K = d_model, both operands K-major); the
+// epilogue stores dH in fp32 (the accumulator as it is).
 // BwdGateUpPair: the recomputed gate/up projection (as FwdHiddenPair, K =
-// d_model) whose epilogue writes, per hidden unit,
-//   SwiGLU: H = SiLU(G) U (bf16), S1 = SiLU(G), S2 = U SiLU'(G)   (fp32)
-//   GeLU:   H = GeLU(G) (bf16),  S1 = GeLU'(G)                     (fp32)
-// DhPair: dH = dY . W_down[c..]^T (K = d_model, both operands K-major) whose
-// epilogue forms the pre-activation gradients from the stored factors,
-//   SwiGLU: dU = dH S1, dG = dH S2;   GeLU: dG = dH S1          (bf16)
-// -- the derivatives of the forward definition, as in BwdHidden; the factors
-// stay fp32 so the only rounding is that of dG / dU, as there.
+// d_model) whose epilogue reads dH and writes, per hidden unit,
+//   SwiGLU: H = SiLU(G) U,  dU = dH SiLU(G),  dG = dH U SiLU'(G)   (bf16)
+//   GeLU:   H = GeLU(G),    dG = dH GeLU'(G)                        (bf16)
+// with SiLU'(g) = s (1 + g (1 - s)), s = sigmoid(g), and GeLU'(z) = Phi(z) +
+// z phi(z): the derivatives of the forward definition.  dH stays fp32, so
+// the only roundings are those of H, dG and dU to bf16.
+struct DhParams {
+    CUtensorMap tmDY;  // dY [n][d], box {64, 128}
+    CUtensorMap tmD;   // W_down / B [f][d], box {64, 128} (K-major: rows are hidden units)
+    int n, d, col_base, width;
+    float* dH;         // [n][width] fp32
+    long long ld;
+};
+
+template <int ACT>
+struct DhPair {
+    using Params = DhParams;
+    static constexpr const char* kName = ACT == 1 ? "bwd_dh_swiglu" : "bwd_dh_gelu";
+    static constexpr int kBK = 64;
+    static constexpr int kABytes = 128 * kBK * 2;
+    static constexpr int kStageBytes = kABytes + 128 * kBK * 2;
+    static constexpr int kStages = 6;
+    static constexpr int kAccCols = 256, kAccBufs = 2;
+    static constexpr uint32_t kIdesc = make_idesc_bf16(256, 256, false, false);
+    struct Tile {
+        int mi, nj;
+    };
+    __host__ __device__ static int num_tiles(const Params& p) {
+        return ((p.n + 255) / 256) * ((p.width + 255) / 256);
+    }
+    __device__ static Tile tile(const Params& p, int t) {
+        const int mt = (p.n + 255) / 256;
+        return Tile{t % mt, t / mt};
+    }
+    __device__ static int num_kb(const Params& p, const Tile&) { return (p.d + kBK - 1) / kBK; }
+    __device__ static void prefetch(const Params& p) {
+        tma_prefetch_desc(&p.tmDY);
+        tma_prefetch_desc(&p.tmD);
+    }
+    __device__ static void load(const Params& p, const Tile& ti, int kb, uint32_t rank, uint32_t st,
+                                uint32_t bar) {
+        const int k0 = kb * kBK;
+        tma_load_2d_pair(st, &p.tmDY, bar, k0, ti.mi * 256 + static_cast<int>(rank) * 128);
+        tma_load_2d_pair(st + kABytes, &p.tmD, bar, k0,
+                         p.col_base + ti.nj * 256 + static_cast<int>(rank) * 128);
+    }
+    __device__ static void mma(const Tile&, int kb, uint32_t st, uint32_t acc) {
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t a = make_smem_desc(st + 32 * kk, 16, 1024, kLayoutSW128);
+            const uint64_t b = make_smem_desc(st + kABytes + 32 * kk, 16, 1024, kLayoutSW128);
+            umma_bf16_pair(acc, a, b, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+        }
+    }
+    __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t rank, uint32_t acc,
+                                    int q, int lane) {
+        const int row = ti.mi * 256 + static_cast<int>(rank) * 128 + q * 32 + lane;
+        const bool row_ok = row < p.n;
+        const long long off = static_cast<long long>(row) * p.ld;
+        const uint32_t t0 = acc + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll 1
+        for (int cc = 0; cc < 8; ++cc) {
+            uint32_t dh[32];
+            tmem_ld_32x32b_x32(t0 + 32 * cc, dh);
+            tmem_ld_wait();
+            const int c0 = ti.nj * 256 + 32 * cc;
+            if (row_ok && c0 < p.width) store_f32x32(p.dH + off + c0, dh, p.width - c0);
+        }
+    }
+};
+
 struct BwdGateUpParams {
     CUtensorMap tmX;  // X [n][d], box {64, 128}
     CUtensorMap tmG;  // W_gate / A [d][f], box {64, 64}
     CUtensorMap tmU;  // W_up [d][f], box {64, 64} (SwiGLU)
     int n, d, col_base, width;
-    __nv_bfloat16* H;  // [n][width]
-    float* S1;         // [n][width]
-    float* S2;         // [n][width] (SwiGLU)
+    const float* dH;     // [n][width] fp32, from DhPair
+    __nv_bfloat16* H;    // [n][width]
+    __nv_bfloat16* dG;   // [n][width]
+    __nv_bfloat16* dU;   // [n][width] (SwiGLU)
     long long ld;
 };
 
@@ -149,6 +215,23 @@ struct BwdGateUpPair {
             umma_bf16_pair(acc, a, b, kIdesc, (kb | kk) != 0 ? 1u : 0u);
         }
     }
+    // 32 fp32 values of dH from src[0..valid) (zero beyond)
+    __device__ static void load_dh(const float* src, int valid, float (&v)[32]) {
+        if (valid >= 32) {
+            const float4* s4 = reinterpret_cast<const float4*>(src);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float4 x = s4[i];
+                v[4 * i] = x.x;
+                v[4 * i + 1] = x.y;
+                v[4 * i + 2] = x.z;
+                v[4 * i + 3] = x.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = i < valid ? src[i] : 0.0f;
+        }
+    }
     __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t rank, uint32_t acc,
                                     int q, int lane) {
         const int row = ti.mi * 256 + static_cast<int>(rank) * 128 + q * 32 + lane;
@@ -157,151 +240,55 @@ struct BwdGateUpPair {
         const uint32_t t0 = acc + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll 1
         for (int cc = 0; cc < (ACT == 1 ? 4 : 8); ++cc) {
-            uint32_t g[32], pk[16], s1[32], s2[32];
+            const int c0 = ti.nj * kOut + 32 * cc;
+            const int valid = p.width - c0;
+            const bool live = row_ok && valid > 0;
+            float dh[32];
+            if (live) load_dh(p.dH + off + c0, valid, dh);
+            uint32_t g[32], ph[16], pg[16], pu[16];
             tmem_ld_32x32b_x32(t0 + 32 * cc, g);
             if (ACT == 1) {
                 uint32_t u[32];
                 tmem_ld_32x32b_x32(t0 + 128 + 32 * cc, u);
                 tmem_ld_wait();
+                if (!live) continue;
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float gv = __uint_as_float(g[i]), uv = __uint_as_float(u[i]);
-                    const float sg = 1.0f / (1.0f + __expf(-gv));
-                    const float si = gv * sg;
-                    s1[i] = __float_as_uint(si);
-                    s2[i] = __float_as_uint(uv * sg * (1.0f + gv * (1.0f - sg)));
-                    g[i] = __float_as_uint(si * uv);
+                for (int i = 0; i < 16; ++i) {
+                    float h[2], dgv[2], duv[2];
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const float gv = __uint_as_float(g[2 * i + j]), uv = __uint_as_float(u[2 * i + j]);
+                        const float sg = 1.0f / (1.0f + __expf(-gv));
+                        const float si = gv * sg;
+                        h[j] = si * uv;
+                        duv[j] = dh[2 * i + j] * si;
+                        dgv[j] = dh[2 * i + j] * (uv * sg * (1.0f + gv * (1.0f - sg)));
+                    }
+                    ph[i] = pack_bf16x2(h[0], h[1]);
+                    pg[i] = pack_bf16x2(dgv[0], dgv[1]);
+                    pu[i] = pack_bf16x2(duv[0], duv[1]);
                 }
+                store_bf16x32(p.dU + off + c0, pu, valid);
             } else {
                 tmem_ld_wait();
+                if (!live) continue;
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float z = __uint_as_float(g[i]);
-                    const float cdf = 0.5f * (1.0f + erff(z * 0.70710678118654752440f));
-                    const float pdf = 0.39894228040143267794f * __expf(-0.5f * z * z);
-                    s1[i] = __float_as_uint(cdf + z * pdf);
-                    g[i] = __float_as_uint(z * cdf);
-                }
-            }
+                for (int i = 0; i < 16; ++i) {
+                    float h[2], dgv[2];
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-                pk[i] = pack_bf16x2(__uint_as_float(g[2 * i]), __uint_as_float(g[2 * i + 1]));
-            const int c0 = ti.nj * kOut + 32 * cc;
-            if (row_ok) {
-                store_bf16x32(p.H + off + c0, pk, p.width - c0);
-                store_f32x32(p.S1 + off + c0, s1, p.width - c0);
-                if (ACT == 1) store_f32x32(p.S2 + off + c0, s2, p.width - c0);
-            }
-        }
-    }
-};
-
-struct DhParams {
-    CUtensorMap tmDY;  // dY [n][d], box {64, 128}
-    CUtensorMap tmD;   // W_down / B [f][d], box {64, 128} (K-major: rows are hidden units)
-    int n, d, col_base, width;
-    const float* S1;   // [n][width]
-    const float* S2;   // [n][width] (SwiGLU)
-    __nv_bfloat16* dG; // [n][width]
-    __nv_bfloat16* dU; // [n][width] (SwiGLU)
-    long long ld;
-};
-
-template <int ACT>
-struct DhPair {
-    using Params = DhParams;
-    static constexpr const char* kName = ACT == 1 ? "bwd_dh_swiglu" : "bwd_dh_gelu";
-    static constexpr int kBK = 64;
-    static constexpr int kABytes = 128 * kBK * 2;
-    static constexpr int kStageBytes = kABytes + 128 * kBK * 2;
-    static constexpr int kStages = 6;
-    static constexpr int kAccCols = 256, kAccBufs = 2;
-    static constexpr uint32_t kIdesc = make_idesc_bf16(256, 256, false, false);
-    struct Tile {
-        int mi, nj;
-    };
-    __host__ __device__ static int num_tiles(const Params& p) {
-        return ((p.n + 255) / 256) * ((p.width + 255) / 256);
-    }
-    __device__ static Tile tile(const Params& p, int t) {
-        const int mt = (p.n + 255) / 256;
-        return Tile{t % mt, t / mt};
-    }
-    __device__ static int num_kb(const Params& p, const Tile&) { return (p.d + kBK - 1) / kBK; }
-    __device__ static void prefetch(const Params& p) {
-        tma_prefetch_desc(&p.tmDY);
-        tma_prefetch_desc(&p.tmD);
-    }
-    __device__ static void load(const Params& p, const Tile& ti, int kb, uint32_t rank, uint32_t st,
-                                uint32_t bar) {
-        const int k0 = kb * kBK;
-        tma_load_2d_pair(st, &p.tmDY, bar, k0, ti.mi * 256 + static_cast<int>(rank) * 128);
-        tma_load_2d_pair(st + kABytes, &p.tmD, bar, k0,
-                         p.col_base + ti.nj * 256 + static_cast<int>(rank) * 128);
-    }
-    __device__ static void mma(const Tile&, int kb, uint32_t st, uint32_t acc) {
-#pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t a = make_smem_desc(st + 32 * kk, 16, 1024, kLayoutSW128);
-            const uint64_t b = make_smem_desc(st + kABytes + 32 * kk, 16, 1024, kLayoutSW128);
-            umma_bf16_pair(acc, a, b, kIdesc, (kb | kk) != 0 ? 1u : 0u);
-        }
-    }
-    __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t rank, uint32_t acc,
-                                    int q, int lane) {
-        const int row = ti.mi * 256 + static_cast<int>(rank) * 128 + q * 32 + lane;
-        const bool row_ok = row < p.n;
-        const long long off = static_cast<long long>(row) * p.ld;
-        const uint32_t t0 = acc + (static_cast<uint32_t>(q * 32) << 16);
-#pragma unroll 1
-        for (int cc = 0; cc < 8; ++cc) {
-            uint32_t dh[32], pg[16], pu[16];
-            tmem_ld_32x32b_x32(t0 + 32 * cc, dh);
-            tmem_ld_wait();
-            const int c0 = ti.nj * 256 + 32 * cc;
-            const int valid = p.width - c0;
-            if (!row_ok || valid <= 0) continue;
-            float f1[32], f2[32];
-            if (valid >= 32) {
-                const float4* a4 = reinterpret_cast<const float4*>(p.S1 + off + c0);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float4 v = a4[i];
-                    f1[4 * i] = v.x;
-                    f1[4 * i + 1] = v.y;
-                    f1[4 * i + 2] = v.z;
-                    f1[4 * i + 3] = v.w;
-                }
-                if (ACT == 1) {
-                    const float4* b4 = reinterpret_cast<const float4*>(p.S2 + off + c0);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const float4 v = b4[i];
-                        f2[4 * i] = v.x;
-                        f2[4 * i + 1] = v.y;
-                        f2[4 * i + 2] = v.z;
-                        f2[4 * i + 3] = v.w;
+                    for (int j = 0; j < 2; ++j) {
+                        const float z = __uint_as_float(g[2 * i + j]);
+                        const float cdf = 0.5f * (1.0f + erff(z * 0.70710678118654752440f));
+                        const float pdf = 0.39894228040143267794f * __expf(-0.5f * z * z);
+                        h[j] = z * cdf;
+                        dgv[j] = dh[2 * i + j] * (cdf + z * pdf);
                     }
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    f1[i] = i < valid ? p.S1[off + c0 + i] : 0.f;
-                    f2[i] = (ACT == 1 && i < valid) ? p.S2[off + c0 + i] : 0.f;
+                    ph[i] = pack_bf16x2(h[0], h[1]);
+                    pg[i] = pack_bf16x2(dgv[0], dgv[1]);
                 }
             }
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const float a0 = __uint_as_float(dh[2 * i]), a1 = __uint_as_float(dh[2 * i + 1]);
-                if (ACT == 1) {
-                    pu[i] = pack_bf16x2(a0 * f1[2 * i], a1 * f1[2 * i + 1]);
-                    pg[i] = pack_bf16x2(a0 * f2[2 * i], a1 * f2[2 * i + 1]);
-                } else {
-                    pg[i] = pack_bf16x2(a0 * f1[2 * i], a1 * f1[2 * i + 1]);
-                }
-            }
+            store_bf16x32(p.H + off + c0, ph, valid);
             store_bf16x32(p.dG + off + c0, pg, valid);
-            if (ACT == 1) store_bf16x32(p.dU + off + c0, pu, valid);
         }
     }
 };

@@ -290,15 +290,22 @@ struct DownAccumPair {
         const int k = (kb - seg * nkb1) * kBK;
         const CUtensorMap* ta = seg ? &p.tmA1 : &p.tmA0;
         const CUtensorMap* tb = seg ? &p.tmB1 : &p.tmB0;
-        tma_load_2d_pair(st, ta, bar, k, ti.s * p.g.seg_rows + ti.mi * 256 + rank * 128);
-        const int kbase = p.g.shard_col(ti.s);
+        // hidden column of this k-block in H (ka) and in the weights (kw)
+        int ka = k, kw = p.g.shard_col(ti.s) + k;
+        if (p.rot_P > 0) {
+            // H holds every hidden unit; segment s visits the shards in ring
+            // order, starting at shard (seg_begin + s) mod P
+            const int sh = k / p.g.fs;
+            ka = kw = ((p.g.seg_begin + ti.s + sh) % p.rot_P) * p.g.fs + (k - sh * p.g.fs);
+        }
+        tma_load_2d_pair(st, ta, bar, ka, ti.s * p.g.seg_rows + ti.mi * 256 + rank * 128);
         const int n0 = ti.nj * BN + static_cast<int>(rank) * kHalf;
         if (B_MN) {
 #pragma unroll
             for (int i = 0; i < kHalf / 64; ++i)
-                tma_load_2d_pair(st + kABytes + 8192 * i, tb, bar, n0 + 64 * i, kbase + k);
+                tma_load_2d_pair(st + kABytes + 8192 * i, tb, bar, n0 + 64 * i, kw);
         } else {
-            tma_load_2d_pair(st + kABytes, tb, bar, kbase + k, n0);
+            tma_load_2d_pair(st + kABytes, tb, bar, kw, n0);
         }
     }
     __device__ static void mma(const Tile&, int kb, uint32_t st, uint32_t acc) {

@@ -206,6 +206,8 @@ struct DownAccum {
         int kdim;         // hidden columns per K-segment
         int n_out;        // output columns
         int mode;
+        int rot_P;        // > 0 (paired kernel): K covers all rot_P shards of g.fs columns,
+                          // segment s starting at shard (seg_begin + s) mod rot_P
         float* acc;       // [rows][n_out] fp32 accumulator (global rows)
         long long ldacc;
         __nv_bfloat16* out;  // [rows][n_out] bf16 (global rows)

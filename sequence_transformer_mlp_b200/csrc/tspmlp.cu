@@ -387,6 +387,9 @@ tsp_status_t validate_backward(const void* X, const void* Wg, const void* Wu, co
 struct FwdPlan {
     bool ok = true;
     bool ring = false;
+    // TSP ring as whole-d_ff hidden blocks per sequence shard and a down
+    // projection with each shard's K loop in ring order (bf16)
+    bool ring_rotated = false;
     // the pass schedule in one paired launch (two H chunk buffers)
     bool fused_passes = false;
     // fused single-launch schedule (bf16)
@@ -446,6 +449,18 @@ FwdPlan plan_forward_budget(int64_t n, int64_t d, int64_t f, int P, tsp_dtype_t 
     }
     if (sched == TSP_SCHED_TSP_RING) {
         pl.ring = true;
+        // bf16 with 64-column shards: each sequence shard's hidden block for all
+        // d_ff columns, and one down projection whose K loop visits the shards in
+        // its ring order (no fp32 accumulator), for as many sequence shards a
+        // launch as fit the budget
+        const size_t per_seg_all = static_cast<size_t>(n / P) * f * e;
+        if (dt == TSP_DT_BF16 && fs % 64 == 0 && budget >= per_seg_all) {
+            pl.ring_rotated = true;
+            pl.tsp_group = static_cast<int>(std::min<size_t>(P, budget / per_seg_all));
+            pl.h_bytes = static_cast<size_t>(pl.tsp_group) * per_seg_all;
+            pl.acc_bytes = 0;
+            return pl;
+        }
         const size_t per_seg = static_cast<size_t>(n / P) * fs * e;
         pl.tsp_group = dt == TSP_DT_BF16
                            ? static_cast<int>(std::min<size_t>(P, budget / std::max<size_t>(per_seg, 1)))
@@ -511,6 +526,11 @@ FwdPlan plan_forward_for(int64_t n, int64_t d, int64_t f, int P, tsp_dtype_t dt,
         if (pl.total() > ws_bytes) pl.ok = false;
         return pl;
     }
+    if (sched == TSP_SCHED_TSP_RING) {
+        // fewer sequence shards a launch, still without an accumulator
+        FwdPlan r = plan_forward_budget(n, d, f, P, dt, sched, ws_bytes);
+        if (r.ring_rotated && r.ok && r.total() <= ws_bytes) return r;
+    }
     const size_t acc = align256(static_cast<size_t>(n) * d * 4);
     if (sched == TSP_SCHED_SHARD_PASSES_FUSED) {
         // two H chunk buffers and the counters
@@ -565,7 +585,7 @@ template <int ACT>
 tsp_status_t fwd_pass_bf16(const void* X, const void* Wg, const void* Wu, const void* Wd,
                            int64_t n, int64_t d, int64_t f, const SegGeom& g, int64_t width,
                            int mode, __nv_bfloat16* H, float* acc, void* Y, cudaStream_t st,
-                           int dev, int sms) {
+                           int dev, int sms, int rot_P = 0) {
     using K1 = FwdHidden<ACT>;
     using K2 = DownAccum<true, 1>;
     typename K1::Params p1;
@@ -591,6 +611,7 @@ tsp_status_t fwd_pass_bf16(const void* X, const void* Wg, const void* Wu, const 
     p2.kdim = static_cast<int>(width);
     p2.n_out = static_cast<int>(d);
     p2.mode = mode;
+    p2.rot_P = rot_P;
     p2.acc = acc;
     p2.ldacc = d;
     p2.out = static_cast<__nv_bfloat16*>(Y);
@@ -764,6 +785,16 @@ tsp_status_t forward_bf16(const void* X, const void* Wg, const void* Wu, const v
             TSP_TRY(fwd_pass_bf16<ACT>(X, Wg, Wu, Wd, n, d, f, g, pl.chunks[i].width,
                                        accum_mode(i, np), H, acc, Y, st, dev, sms));
         }
+    } else if (pl.ring_rotated) {
+        for (int s0 = 0; s0 < P; s0 += pl.tsp_group) {
+            const int cnt = std::min(pl.tsp_group, P - s0);
+            SegGeom g = seg_all_rows(n, P, fs, 0);
+            g.seg_rows = static_cast<int>(n / P);
+            g.num_segs = cnt;
+            g.seg_begin = s0;
+            TSP_TRY(fwd_pass_bf16<ACT>(X, Wg, Wu, Wd, n, d, f, g, f, /*mode direct*/ 3, H, nullptr, Y,
+                                       st, dev, sms, P));
+        }
     } else {
         for (int t = 0; t < P; ++t)
             for (int s0 = 0; s0 < P; s0 += pl.tsp_group) {
@@ -843,7 +874,7 @@ tsp_status_t forward_f32(const float* X, const float* Wg, const float* Wu, const
 struct BwdPlan {
     bool ok = true;
     std::vector<Chunk> chunks;
-    int n16 = 3, n32 = 2;     // bf16 buffers (H, dG, dU) and fp32 factor buffers (S1, S2)
+    int n16 = 3, n32 = 1;     // bf16 buffers (H, dG, dU) and the fp32 dH buffer
     size_t b16 = 0, b32 = 0;  // bytes of one bf16 / fp32 chunk buffer
     size_t acc_bytes = 0;
     size_t total() const {
@@ -854,7 +885,7 @@ struct BwdPlan {
 BwdPlan plan_backward_budget(int64_t n, int64_t d, int64_t f, int P, tsp_act_t act, size_t budget) {
     BwdPlan pl;
     pl.n16 = act == TSP_ACT_SWIGLU ? 3 : 2;
-    pl.n32 = act == TSP_ACT_SWIGLU ? 2 : 1;
+    pl.n32 = 1;
     const size_t per_col = static_cast<size_t>(n) * (2 * pl.n16 + 4 * pl.n32);
     const int64_t mc = max_chunk_cols(budget, per_col);
     if (mc == 0) {
@@ -897,14 +928,28 @@ tsp_status_t backward_bf16(const void* X, const void* Wg, const void* Wu, const 
     auto* Hc = reinterpret_cast<__nv_bfloat16*>(w);
     auto* dGc = reinterpret_cast<__nv_bfloat16*>(w + a16);
     auto* dUc = ACT == 1 ? reinterpret_cast<__nv_bfloat16*>(w + 2 * a16) : nullptr;
-    auto* S1 = reinterpret_cast<float*>(w + pl.n16 * a16);
-    auto* S2 = ACT == 1 ? reinterpret_cast<float*>(w + pl.n16 * a16 + a32) : nullptr;
+    auto* dHc = reinterpret_cast<float*>(w + pl.n16 * a16);
     float* acc = pl.acc_bytes ? reinterpret_cast<float*>(w + pl.n16 * a16 + pl.n32 * a32) : nullptr;
     const int64_t fs = f / P;
     const int np = static_cast<int>(pl.chunks.size());
     for (int i = 0; i < np; ++i) {
         const int64_t cb = pl.chunks[i].col_base, C = pl.chunks[i].width;
-        // K3a: recompute G (U); emit H and the activation-derivative factors
+        // K3a: dH = dY . W_down[chunk]^T, kept in fp32
+        {
+            DhParams p;
+            std::memset(&p, 0, sizeof(p));
+            if (!tmap_bf16(&p.tmDY, dY, d, n, d, 64, 128, SW128) ||
+                !tmap_bf16(&p.tmD, Wd, d, f, d, 64, 128, SW128))
+                return TSP_ERR_CUDA;
+            p.n = static_cast<int>(n);
+            p.d = static_cast<int>(d);
+            p.col_base = static_cast<int>(cb);
+            p.width = static_cast<int>(C);
+            p.dH = dHc;
+            p.ld = C;
+            TSP_TRY(launch_pair<DhPair<ACT>>(p, st, dev, sms));
+        }
+        // K3b: recompute G (U); emit H and, from dH, dG (dU)
         {
             BwdGateUpParams p;
             std::memset(&p, 0, sizeof(p));
@@ -916,29 +961,12 @@ tsp_status_t backward_bf16(const void* X, const void* Wg, const void* Wu, const 
             p.d = static_cast<int>(d);
             p.col_base = static_cast<int>(cb);
             p.width = static_cast<int>(C);
+            p.dH = dHc;
             p.H = Hc;
-            p.S1 = S1;
-            p.S2 = S2;
-            p.ld = C;
-            TSP_TRY(launch_pair<BwdGateUpPair<ACT>>(p, st, dev, sms));
-        }
-        // K3b: dH = dY . W_down[chunk]^T; emit dG (dU) from the factors
-        {
-            DhParams p;
-            std::memset(&p, 0, sizeof(p));
-            if (!tmap_bf16(&p.tmDY, dY, d, n, d, 64, 128, SW128) ||
-                !tmap_bf16(&p.tmD, Wd, d, f, d, 64, 128, SW128))
-                return TSP_ERR_CUDA;
-            p.n = static_cast<int>(n);
-            p.d = static_cast<int>(d);
-            p.col_base = static_cast<int>(cb);
-            p.width = static_cast<int>(C);
-            p.S1 = S1;
-            p.S2 = S2;
             p.dG = dGc;
             p.dU = dUc;
             p.ld = C;
-            TSP_TRY(launch_pair<DhPair<ACT>>(p, st, dev, sms));
+            TSP_TRY(launch_pair<BwdGateUpPair<ACT>>(p, st, dev, sms));
         }
         // K4a: dW_down[cb .. cb+C) = H^T . dY
         {

@@ -87,6 +87,11 @@ def test_workspace_sizes_follow_the_schedule(lib):
     # TSP ring passes: sequence shards per launch within the hidden budget + accumulator
     wsr = T.tsp_mlp_workspace_size(32768, d, f, P, "swiglu", "bf16", "tsp_ring_fused")
     assert wsr == _a256(24 * 128 * f * 2) + _a256((1 + 2 * 256) * 4)
+    # TSP ring passes with 64-multiple shards: whole-d_ff hidden blocks of as
+    # many sequence shards as fit 512 MB (4 of 117 MB), no accumulator
+    assert T.tsp_mlp_workspace_size(32768, d, f, P, "swiglu", "bf16", "tsp_ring") == \
+        4 * 4096 * f * 2
+    # ... otherwise one ring step's shard blocks within the budget + the accumulator
     wsr2 = T.tsp_mlp_workspace_size(8 * 100, 256, 8 * 96, 8, "swiglu", "bf16", "tsp_ring")
     assert wsr2 == _a256(8 * 100 * 96 * 2) + _a256(800 * 256 * 4)
     # fused schedules need bf16; the fused ring needs 64-multiple shards
@@ -94,8 +99,10 @@ def test_workspace_sizes_follow_the_schedule(lib):
     assert lib.tsp_mlp_workspace_size(64, 64, 128, 1, 1, 1, 3, 0, ctypes.byref(out)) == 2
     assert lib.tsp_mlp_workspace_size(8 * 100, 256, 8 * 96, 8, 1, 0, 4, 0, ctypes.byref(out)) == 2
     # backward: H, dG, dU chunk buffers and the fp32 dX accumulator
+    # backward: bf16 H, dG, dU and fp32 dH for all hidden units (one chunk
+    # within the 1 GiB budget, so no fp32 dX accumulator)
     wsb = T.tsp_mlp_workspace_size(n, d, f, P, "swiglu", "bf16", backward=True)
-    assert wsb > acc
+    assert wsb == 3 * n * f * 2 + n * f * 4
 
 
 @pytest.mark.parametrize("args,code", [

@@ -79,9 +79,9 @@ def test_backward_multi_pass(act):
     n, d, f, P = 384, 256, 4 * 256, 4
     wl = Workload("bwd_mp", act, "bf16", n, d, f, P, seed=5, w_std=0.05, backward=True)
     inp = make_inputs(wl)
-    # bf16 buffers H, dG (dU) and fp32 factor buffers S1 (S2) of one 128-column
-    # chunk each, plus the fp32 dX accumulator
-    n16, n32 = (3, 2) if act == "swiglu" else (2, 1)
+    # bf16 buffers H, dG (dU) and the fp32 dH buffer of one 128-column chunk
+    # each, plus the fp32 dX accumulator
+    n16, n32 = (3, 1) if act == "swiglu" else (2, 1)
     ws = n * d * 4 + 2048 + n16 * (n * 128 * 2 + 256) + n32 * (n * 128 * 4 + 256) + 4096
     dX, dWg, dWu, dWd = gpu_backward(inp, P, act, ws_bytes=ws)
     ref = oracle.mlp_backward(inp["X"], inp["A"], inp["Wu"], inp["B"], inp["dY"], act)

@@ -187,6 +187,7 @@ def test_bf16_independent_of_P(P):
 
 @pytest.mark.parametrize("n,d,f,P,sched", [(4 * 128, 128, 4 * 128, 4, "tsp_ring"),
                                            (8 * 100, 256, 8 * 96, 8, "tsp_ring"),
+                                           (8 * 100, 256, 8 * 128, 8, "tsp_ring"),
                                            (2 * 64, 64, 2 * 64, 2, "tsp_ring"),
                                            (4 * 128, 128, 4 * 128, 4, "tsp_ring_fused"),
                                            (8 * 200, 256, 8 * 128, 8, "tsp_ring_fused"),
@@ -197,6 +198,18 @@ def test_bf16_tsp_ring_small(n, d, f, P, sched):
     Y = gpu_forward(inp, P, "swiglu", sched)
     ref = oracle.mlp_tsp(inp["X"], inp["A"], inp["Wu"], inp["B"], "swiglu", P)
     check(Y, ref, "bf16", "tsp ring")
+
+
+def test_bf16_tsp_ring_sequence_shard_groups():
+    """A workspace with room for two sequence shards' hidden blocks: the ring
+    runs as two launches of two shards, each shard's K loop in its ring order."""
+    n, d, f, P = 4 * 128, 128, 4 * 128, 4
+    wl = small("swiglu", "bf16", n, d, f, P, seed=12)
+    inp = make_inputs(wl)
+    ws = 2 * (n // P) * f * 2 + 256
+    Y = gpu_forward(inp, P, "swiglu", "tsp_ring", ws_bytes=ws)
+    ref = oracle.mlp_tsp(inp["X"], inp["A"], inp["Wu"], inp["B"], "swiglu", P)
+    check(Y, ref, "bf16", "tsp ring, 2 shards a launch")
 
 
 @pytest.mark.parametrize("sched", ["weight_shards", "shard_passes_fused", "fused", "tsp_ring",

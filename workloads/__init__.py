@@ -66,7 +66,7 @@ WORKLOADS = {
                                                4096, 4096, 14336, 8, seed=1, w_std=0.02),
     "tsp_ring_bf16_n32768_d4096_f14336": Workload("tsp_ring_bf16_n32768_d4096_f14336", "swiglu",
                                                   "bf16", 32768, 4096, 14336, 8, seed=2,
-                                                  w_std=0.02, sched="tsp_ring_fused"),
+                                                  w_std=0.02, sched="tsp_ring"),
     "swiglu_bf16_n8192_d8192_f28672": Workload("swiglu_bf16_n8192_d8192_f28672", "swiglu", "bf16",
                                                8192, 8192, 28672, 8, seed=3, w_std=0.015),
     "swiglu_bf16_fwdbwd_n4096_d4096_f14336": Workload("swiglu_bf16_fwdbwd_n4096_d4096_f14336",
