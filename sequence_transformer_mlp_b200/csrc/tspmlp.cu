@@ -40,6 +40,11 @@ constexpr int kMaxDevices = 64;
 // (or two H chunk buffers) within L2-sized budgets: their consumers read H
 // while it is being produced.
 constexpr size_t kFwdHiddenBudget = 512ull << 20;  // one bf16 [rows][C] buffer
+// The rotated TSP ring's sequence shards a launch, and the token rows a
+// one-chunk pass takes: the down projection reads the group's H while that is
+// still in L2.
+constexpr size_t kRingGroupBudget = 512ull << 20;
+constexpr size_t kRowGroupBudget = 128ull << 20;
 constexpr size_t kFusedRingBudget = 96ull << 20;   // the fused schedule's H ring
 constexpr size_t kFusedPassesBudget = 128ull << 20; // two H chunk buffers of the one-launch passes
 // H, dG, dU (bf16) and the fp32 activation-derivative factors together.  The
@@ -399,6 +404,7 @@ struct FwdPlan {
     // per-chunk pass schedule
     std::vector<Chunk> chunks;  // weight-shard passes
     int tsp_group = 1;          // ring passes: sequence shards per launch
+    int64_t row_group = 0;      // > 0: one-chunk passes over groups of this many token rows
     size_t h_bytes = 0, acc_bytes = 0;
     size_t total() const {
         if (fused) return align256(ring_bytes) + align256(sync_bytes);
@@ -456,7 +462,8 @@ FwdPlan plan_forward_budget(int64_t n, int64_t d, int64_t f, int P, tsp_dtype_t 
         const size_t per_seg_all = static_cast<size_t>(n / P) * f * e;
         if (dt == TSP_DT_BF16 && fs % 64 == 0 && budget >= per_seg_all) {
             pl.ring_rotated = true;
-            pl.tsp_group = static_cast<int>(std::min<size_t>(P, budget / per_seg_all));
+            pl.tsp_group = static_cast<int>(
+                std::min<size_t>(P, std::max<size_t>(1, std::min(budget, kRingGroupBudget) / per_seg_all)));
             pl.h_bytes = static_cast<size_t>(pl.tsp_group) * per_seg_all;
             pl.acc_bytes = 0;
             return pl;
@@ -472,6 +479,23 @@ FwdPlan plan_forward_budget(int64_t n, int64_t d, int64_t f, int P, tsp_dtype_t 
         pl.h_bytes = static_cast<size_t>(pl.tsp_group) * per_seg;
         pl.acc_bytes = (dt == TSP_DT_BF16 && P > 1) ? static_cast<size_t>(n) * d * 4 : 0;
         return pl;
+    }
+    if (dt == TSP_DT_BF16 && sched != TSP_SCHED_SHARD_PASSES_FUSED) {
+        // Row groups: token rows are independent, so when all of H does not
+        // fit in L2 the rows run in equal groups (multiples of 256) of at
+        // most kRowGroupBudget of H, each a one-chunk pass summing every shard
+        // in tensor memory -- no fp32 accumulator, H read back from L2.
+        const size_t per_row = static_cast<size_t>(f) * e;
+        const size_t rg = std::min(budget, kRowGroupBudget);
+        const int64_t cap = static_cast<int64_t>(rg / per_row) / 256 * 256;
+        if (static_cast<size_t>(n) * per_row > rg && cap >= 256) {
+            const int64_t groups = (n + cap - 1) / cap;
+            pl.row_group = ((n + groups - 1) / groups + 255) / 256 * 256;
+            pl.chunks = {{0, f}};
+            pl.h_bytes = static_cast<size_t>(pl.row_group) * per_row;
+            pl.acc_bytes = 0;
+            return pl;
+        }
     }
     if (dt == TSP_DT_BF16) {
         // the one-launch pass schedule holds two H chunks; it needs chunk widths
@@ -526,10 +550,11 @@ FwdPlan plan_forward_for(int64_t n, int64_t d, int64_t f, int P, tsp_dtype_t dt,
         if (pl.total() > ws_bytes) pl.ok = false;
         return pl;
     }
-    if (sched == TSP_SCHED_TSP_RING) {
-        // fewer sequence shards a launch, still without an accumulator
+    {
+        // fewer sequence shards (ring) or token rows (row groups) a launch,
+        // still without an accumulator
         FwdPlan r = plan_forward_budget(n, d, f, P, dt, sched, ws_bytes);
-        if (r.ring_rotated && r.ok && r.total() <= ws_bytes) return r;
+        if ((r.ring_rotated || r.row_group > 0) && r.ok && r.total() <= ws_bytes) return r;
     }
     const size_t acc = align256(static_cast<size_t>(n) * d * 4);
     if (sched == TSP_SCHED_SHARD_PASSES_FUSED) {
@@ -778,6 +803,19 @@ tsp_status_t forward_bf16(const void* X, const void* Wg, const void* Wu, const v
                                                          align256(pl.h_bytes))
                               : nullptr;
     const int64_t fs = f / P;
+    if (pl.row_group > 0) {
+        // independent row groups: each a complete one-chunk pass on offset views
+        const size_t xe = static_cast<size_t>(d) * 2;
+        for (int64_t r0 = 0; r0 < n; r0 += pl.row_group) {
+            const int64_t rows = std::min<int64_t>(pl.row_group, n - r0);
+            const void* Xg = static_cast<const char*>(X) + r0 * xe;
+            void* Yg = static_cast<char*>(Y) + r0 * xe;
+            const SegGeom g = seg_all_rows(rows, P, fs, 0);
+            TSP_TRY(fwd_pass_bf16<ACT>(Xg, Wg, Wu, Wd, rows, d, f, g, f, 3, H, nullptr, Yg, st, dev,
+                                       sms));
+        }
+        return TSP_OK;
+    }
     if (!pl.ring) {
         const int np = static_cast<int>(pl.chunks.size());
         for (int i = 0; i < np; ++i) {

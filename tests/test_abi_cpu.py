@@ -75,11 +75,11 @@ def test_workspace_sizes_follow_the_schedule(lib):
     assert ws == T.tsp_mlp_workspace_size(n, d, f, P, "swiglu", "bf16") == n * f * 2
     assert T.tsp_mlp_workspace_size(n, d, f, P, "swiglu", "bf16", "shard_passes_fused") == \
         2 * (n * f // 2 * 2) + acc + _a256((1 + 2 * 2 * 16) * 4)
-    # 70B shape: 470 MB of H in one chunk; 32768 tokens of the 8B shape: 940 MB
-    # of H in two chunks of four shards + the accumulator
-    assert T.tsp_mlp_workspace_size(8192, 8192, 28672, 8, "swiglu", "bf16") == 8192 * 28672 * 2
-    assert T.tsp_mlp_workspace_size(32768, d, f, P, "swiglu", "bf16") == \
-        32768 * (f // 2) * 2 + 32768 * d * 4
+    # H larger than the 128 MB row-group budget: equal groups of token rows
+    # (multiples of 256), each a one-chunk pass -- 70B shape: 4 groups of 2048
+    # rows; 32768 tokens of the 8B shape: 8 groups of 4096 rows
+    assert T.tsp_mlp_workspace_size(8192, 8192, 28672, 8, "swiglu", "bf16") == 2048 * 28672 * 2
+    assert T.tsp_mlp_workspace_size(32768, d, f, P, "swiglu", "bf16") == 4096 * f * 2
     # single chunk: no accumulator
     assert T.tsp_mlp_workspace_size(256, 64, 512, 1, "swiglu", "bf16", "shard_passes") == \
         256 * 512 * 2

@@ -200,6 +200,17 @@ def test_bf16_tsp_ring_small(n, d, f, P, sched):
     check(Y, ref, "bf16", "tsp ring")
 
 
+def test_bf16_row_groups_from_a_small_workspace():
+    """A workspace with room for 512 rows of H: the forward runs as two
+    one-chunk passes over token rows 0-511 and 512-999 (a ragged last group)."""
+    n, d, f, P = 1000, 256, 4 * 256, 4
+    wl = small("swiglu", "bf16", n, d, f, P, seed=13)
+    inp = make_inputs(wl)
+    Y = gpu_forward(inp, P, "swiglu", "weight_shards", ws_bytes=512 * f * 2)
+    ref = oracle.mlp_forward(inp["X"], inp["A"], inp["Wu"], inp["B"], "swiglu")
+    check(Y, ref, "bf16", "row groups of 512")
+
+
 def test_bf16_tsp_ring_sequence_shard_groups():
     """A workspace with room for two sequence shards' hidden blocks: the ring
     runs as two launches of two shards, each shard's K loop in its ring order."""
