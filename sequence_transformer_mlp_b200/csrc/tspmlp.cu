@@ -164,32 +164,6 @@ void trace_end(cudaStream_t st, TraceRec* rec) {
 // ---------------------------------------------------------------------------
 // launches
 
-template <class R>
-tsp_status_t launch_umma(const typename R::Params& p, cudaStream_t st, int dev, int sms) {
-    const int tiles = R::num_tiles(p);
-    if (tiles <= 0) return TSP_OK;
-    constexpr int smem = pipeline_smem_bytes<R>();
-    static_assert(smem <= 232448, "stage ring exceeds 227 KB of shared memory");
-    static bool attr_set[kMaxDevices] = {};
-    {
-        std::lock_guard<std::mutex> lk(g_mu);
-        if (!attr_set[dev]) {
-            if (cudaFuncSetAttribute(umma_pipeline_kernel<R>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     smem) != cudaSuccess)
-                return TSP_ERR_CUDA;
-            attr_set[dev] = true;
-        }
-    }
-    const int grid = std::min(tiles, sms);
-    TraceRec rec;
-    const bool traced = trace_begin(st, &rec, R::kName);
-    umma_pipeline_kernel<R><<<grid, kPipelineThreads, smem, st>>>(p);
-    const cudaError_t e = cudaGetLastError();
-    if (traced) trace_end(st, &rec);
-    return e == cudaSuccess ? TSP_OK : TSP_ERR_CUDA;
-}
-
 // Paired launch: clusters of two CTAs (cta_group::2 tiles), as many pairs as
 // can be resident at once, each walking the tile list persistently.
 template <class R>
