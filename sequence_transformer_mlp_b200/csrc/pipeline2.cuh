@@ -285,8 +285,11 @@ struct DownAccumPair {
     __device__ static void prefetch(const Params& p) { Base::prefetch(p); }
     __device__ static void load(const Params& p, const Tile& ti, int kb, uint32_t rank, uint32_t st,
                                 uint32_t bar) {
+        // K segment of this k-block (NSEG <= 2), without a division: this runs
+        // once per k-block in the producer thread
+        static_assert(NSEG == 1 || NSEG == 2, "one or two K segments");
         const int nkb1 = (p.kdim + kBK - 1) / kBK;
-        const int seg = NSEG > 1 ? kb / nkb1 : 0;
+        const int seg = (NSEG > 1 && kb >= nkb1) ? 1 : 0;
         const int k = (kb - seg * nkb1) * kBK;
         const CUtensorMap* ta = seg ? &p.tmA1 : &p.tmA0;
         const CUtensorMap* tb = seg ? &p.tmB1 : &p.tmB0;
@@ -294,9 +297,13 @@ struct DownAccumPair {
         int ka = k, kw = p.g.shard_col(ti.s) + k;
         if (p.rot_P > 0) {
             // H holds every hidden unit; segment s visits the shards in ring
-            // order, starting at shard (seg_begin + s) mod P
-            const int sh = k / p.g.fs;
-            ka = kw = ((p.g.seg_begin + ti.s + sh) % p.rot_P) * p.g.fs + (k - sh * p.g.fs);
+            // order, starting at shard seg_begin + s (< P): column k of the
+            // loop is hidden unit (k + (seg_begin + s) fs) mod (P fs).  No
+            // division: this runs once per k-block in the producer thread.
+            const int f_all = p.rot_P * p.g.fs;
+            ka = k + (p.g.seg_begin + ti.s) * p.g.fs;
+            if (ka >= f_all) ka -= f_all;
+            kw = ka;
         }
         tma_load_2d_pair(st, ta, bar, ka, ti.s * p.g.seg_rows + ti.mi * 256 + rank * 128);
         const int n0 = ti.nj * BN + static_cast<int>(rank) * kHalf;
