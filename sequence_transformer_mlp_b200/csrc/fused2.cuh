@@ -242,6 +242,7 @@ __global__ void __launch_bounds__(kPipelineThreads, 1)
                     nkb = nkb_up;
                 }
                 const int row = ti.m * 256 + static_cast<int>(rank) * 128;
+                const int cbase = p.cb[ti.c];  // read once a tile, not per k-block
                 bool ok = true;
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) {
@@ -254,7 +255,7 @@ __global__ void __launch_bounds__(kPipelineThreads, 1)
                     const int k0 = kb * Cfg::kBK;
                     if (ti.type == 0) {
                         tma_load_2d_pair(st, &p.tmX, fb, k0, row);
-                        const int c = p.cb[ti.c] + ti.j * Cfg::kOut;
+                        const int c = cbase + ti.j * Cfg::kOut;
                         if (ACT == 1) {
                             const CUtensorMap* w = leader ? &p.tmG : &p.tmU;
                             tma_load_2d_pair(st + Cfg::kABytes, w, fb, c, k0);
@@ -267,9 +268,8 @@ __global__ void __launch_bounds__(kPipelineThreads, 1)
                     } else {
                         tma_load_2d_pair(st, (ti.c & 1) ? &p.tmH1 : &p.tmH0, fb, k0, row);
                         const int n0 = ti.j * 256 + static_cast<int>(rank) * 128;
-                        tma_load_2d_pair(st + Cfg::kABytes, &p.tmD, fb, n0, p.cb[ti.c] + k0);
-                        tma_load_2d_pair(st + Cfg::kABytes + 8192, &p.tmD, fb, n0 + 64,
-                                         p.cb[ti.c] + k0);
+                        tma_load_2d_pair(st + Cfg::kABytes, &p.tmD, fb, n0, cbase + k0);
+                        tma_load_2d_pair(st + Cfg::kABytes + 8192, &p.tmD, fb, n0 + 64, cbase + k0);
                     }
                     armed |= 1u << stage;
                     armed_par = (armed_par & ~(1u << stage)) | (phase << stage);

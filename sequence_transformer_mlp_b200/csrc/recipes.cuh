@@ -198,6 +198,8 @@ struct FwdHidden {
 // A is K-major (hidden activations, [rows][kdim]); B is MN-major (W_down
 // [f][d], forward) or K-major (W_gate / W_up [d][f], input gradient).
 // Modes: 0 store fp32, 1 add into fp32, 2 bf16(acc + tile) to out, 3 bf16(tile).
+// This struct holds the launch parameters and the per-row epilogue; the
+// paired kernel (DownAccumPair in pipeline2.cuh) does the loads and MMAs.
 template <bool B_MN, int NSEG>
 struct DownAccum {
     struct Params {
@@ -215,30 +217,6 @@ struct DownAccum {
     };
     static constexpr const char* kName =
         B_MN ? "down_accum_fwd" : (NSEG == 2 ? "dgrad_accum_swiglu" : "dgrad_accum_gelu");
-    static constexpr int kBK = 64;
-    static constexpr int kABytes = 128 * kBK * 2;
-    static constexpr int kBBytes = 256 * kBK * 2;
-    static constexpr int kStageBytes = kABytes + kBBytes;
-    static constexpr int kStages = 4;
-    static constexpr int kAccCols = 256, kAccBufs = 2, kTmemCols = 512;
-    static constexpr uint32_t kIdesc = make_idesc_bf16(128, 256, false, B_MN);
-    struct Tile {
-        int s, mi, nj;
-    };
-    __host__ __device__ static int ntiles_n(const Params& p) { return (p.n_out + 255) / 256; }
-    __host__ __device__ static int num_tiles(const Params& p) {
-        return p.g.num_segs * p.g.mtiles() * ntiles_n(p);
-    }
-    // segment-major, then output slab, then row tile (row tiles fastest): one
-    // sequence segment's rows and weight shard at a time stay in L2
-    __device__ static Tile tile(const Params& p, int t) {
-        const int mt = p.g.mtiles(), per_seg = mt * ntiles_n(p);
-        const int s = t / per_seg, r = t - s * per_seg;
-        return Tile{s, r % mt, r / mt};
-    }
-    __device__ static int num_kb(const Params& p, const Tile&) {
-        return NSEG * ((p.kdim + kBK - 1) / kBK);
-    }
     __device__ static void prefetch(const Params& p) {
         tma_prefetch_desc(&p.tmA0);
         tma_prefetch_desc(&p.tmB0);
@@ -246,36 +224,6 @@ struct DownAccum {
             tma_prefetch_desc(&p.tmA1);
             tma_prefetch_desc(&p.tmB1);
         }
-    }
-    __device__ static uint32_t load_bytes(const Params&, const Tile&, int) { return kStageBytes; }
-    __device__ static void load(const Params& p, const Tile& ti, int kb, uint32_t st, uint32_t bar) {
-        const int nkb1 = (p.kdim + kBK - 1) / kBK;
-        const int seg = NSEG > 1 ? kb / nkb1 : 0;
-        const int k = (kb - seg * nkb1) * kBK;
-        const CUtensorMap* ta = seg ? &p.tmA1 : &p.tmA0;
-        const CUtensorMap* tb = seg ? &p.tmB1 : &p.tmB0;
-        tma_load_2d(st, ta, bar, k, ti.s * p.g.seg_rows + ti.mi * 128);
-        const int kbase = p.g.shard_col(ti.s);
-        const uint32_t b = st + kABytes;
-        if (B_MN) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) tma_load_2d(b + 8192 * i, tb, bar, ti.nj * 256 + 64 * i, kbase + k);
-        } else {
-            tma_load_2d(b, tb, bar, kbase + k, ti.nj * 256);
-        }
-    }
-    __device__ static void mma(const Tile&, int kb, uint32_t st, uint32_t acc) {
-#pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t a = make_smem_desc(st + 32 * kk, 16, 1024, kLayoutSW128);
-            const uint64_t b = B_MN ? make_smem_desc(st + kABytes + 2048 * kk, 8192, 1024, kLayoutSW128)
-                                    : make_smem_desc(st + kABytes + 32 * kk, 16, 1024, kLayoutSW128);
-            umma_bf16(acc, a, b, kIdesc, (kb | kk) != 0 ? 1u : 0u);
-        }
-    }
-    __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t acc, int q, int lane) {
-        store_rows<8>(p, ti.s, ti.mi * 128 + q * 32 + lane, ti.nj * 256,
-                      acc + (static_cast<uint32_t>(q * 32) << 16));
     }
     // One thread's accumulator row (tile row rl of segment s) over NCHUNK x 32
     // columns starting at output column col0, applied in the launch's mode.
@@ -348,6 +296,8 @@ struct DownAccum {
 //   out[r][c] = sum_tok A[tok][a_col0 + r] * B[tok][b_col0 + c]
 // SPLIT: B is two 128-column sources (dG | dU) written to out0 | out1
 // (dW_gate, dW_up share the X operand); otherwise one source of NCOLS.
+// This struct holds the launch parameters and the per-row epilogue; the
+// paired kernel (WgradPair in bwd_pair.cuh) does the loads and MMAs.
 template <int NCOLS, bool SPLIT>
 struct Wgrad {
     struct Params {
@@ -362,57 +312,14 @@ struct Wgrad {
     };
     static constexpr const char* kName =
         SPLIT ? "wgrad_gate_up" : (NCOLS == 256 ? "wgrad_down" : "wgrad_gelu_a");
-    static constexpr int kBK = 64;
-    static constexpr int kABytes = 128 * kBK * 2;
-    static constexpr int kBBytes = NCOLS * kBK * 2;
-    static constexpr int kStageBytes = kABytes + kBBytes;
-    static constexpr int kStages = kStageBytes <= 32768 ? 6 : 4;
-    static constexpr int kAccCols = 256, kAccBufs = 2, kTmemCols = 512;
     static constexpr int kTileCols = SPLIT ? NCOLS / 2 : NCOLS;
-    static constexpr uint32_t kIdesc = make_idesc_bf16(128, NCOLS, true, true);
     struct Tile {
-        int mi, nj;
+        int mi, nj;  // 128-row block of the output, NCOLS-column block
     };
-    __host__ __device__ static int num_tiles(const Params& p) {
-        return ((p.m_valid + 127) / 128) * ((p.n_valid + kTileCols - 1) / kTileCols);
-    }
-    __device__ static Tile tile(const Params& p, int t) {
-        const int mt = (p.m_valid + 127) / 128;
-        return Tile{t % mt, t / mt};
-    }
-    __device__ static int num_kb(const Params& p, const Tile&) { return (p.ntok + kBK - 1) / kBK; }
     __device__ static void prefetch(const Params& p) {
         tma_prefetch_desc(&p.tmA);
         tma_prefetch_desc(&p.tmB0);
         if (SPLIT) tma_prefetch_desc(&p.tmB1);
-    }
-    __device__ static uint32_t load_bytes(const Params&, const Tile&, int) { return kStageBytes; }
-    __device__ static void load(const Params& p, const Tile& ti, int kb, uint32_t st, uint32_t bar) {
-        const int k0 = kb * kBK;
-        const int a = p.a_col0 + ti.mi * 128;
-        tma_load_2d(st, &p.tmA, bar, a, k0);
-        tma_load_2d(st + 8192, &p.tmA, bar, a + 64, k0);
-        const uint32_t b = st + kABytes;
-        if (SPLIT) {
-            const int c = p.b_col0 + ti.nj * (NCOLS / 2);
-#pragma unroll
-            for (int i = 0; i < NCOLS / 128; ++i) {
-                tma_load_2d(b + 8192 * i, &p.tmB0, bar, c + 64 * i, k0);
-                tma_load_2d(b + 8192 * (i + NCOLS / 128), &p.tmB1, bar, c + 64 * i, k0);
-            }
-        } else {
-            const int c = p.b_col0 + ti.nj * NCOLS;
-#pragma unroll
-            for (int i = 0; i < NCOLS / 64; ++i) tma_load_2d(b + 8192 * i, &p.tmB0, bar, c + 64 * i, k0);
-        }
-    }
-    __device__ static void mma(const Tile&, int kb, uint32_t st, uint32_t acc) {
-#pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t a = make_smem_desc(st + 2048 * kk, 8192, 1024, kLayoutSW128);
-            const uint64_t b = make_smem_desc(st + kABytes + 2048 * kk, 8192, 1024, kLayoutSW128);
-            umma_bf16(acc, a, b, kIdesc, (kb | kk) != 0 ? 1u : 0u);
-        }
     }
     __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t acc, int q, int lane) {
         const int rl = ti.mi * 128 + q * 32 + lane;
