@@ -95,6 +95,10 @@ __global__ void __launch_bounds__(kPipelineThreads, 1)
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0, armed = 0, armed_par = 0;
+            // the leader's full barriers in the cluster window, mapped once
+            // (the barriers are contiguous; checked, else mapped per load)
+            const uint32_t full0_leader = map_to_cta(full_bar(0), 0);
+            const bool linear_map = map_to_cta(full_bar(S - 1), 0) == full0_leader + 8u * (S - 1);
             for (int t = pair; t < num_tiles && !*abort_flag; t += npairs) {
                 const auto ti = R::tile(p, t);
                 const int nkb = R::num_kb(p, ti);
@@ -102,7 +106,7 @@ __global__ void __launch_bounds__(kPipelineThreads, 1)
                     if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) break;
                     if (leader) mbar_arrive_expect_tx(full_bar(stage), 2u * R::kStageBytes);
                     R::load(p, ti, kb, rank, ring + stage * R::kStageBytes,
-                            map_to_cta(full_bar(stage), 0));
+                            linear_map ? full0_leader + 8u * stage : map_to_cta(full_bar(stage), 0));
                     armed |= 1u << stage;
                     armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
                     if (++stage == S) {
@@ -204,6 +208,8 @@ struct FwdHiddenPair {
     static constexpr uint32_t kIdesc = make_idesc_bf16(256, 256, false, true);
     struct Tile {
         int s, mi, nj;
+        int c;     // first weight column of the tile (shard base + nj kOut)
+        int xrow;  // first X row of the pair's 256 rows
     };
     __host__ __device__ static int pair_mtiles(const SegGeom& g) { return (g.seg_rows + 255) >> 8; }
     __host__ __device__ static int ntiles_n(const Params& p) { return (p.width + kOut - 1) / kOut; }
@@ -213,16 +219,18 @@ struct FwdHiddenPair {
     __device__ static Tile tile(const Params& p, int t) {
         const int mt = pair_mtiles(p.g), per_seg = mt * ntiles_n(p);
         const int s = t / per_seg, r = t - s * per_seg;
-        return Tile{s, r % mt, r / mt};
+        const int nj = r / mt;
+        const int mi = r - nj * mt;
+        // everything the per-k-block loads need, computed once a tile
+        return Tile{s, mi, nj, p.g.shard_col(s) + nj * kOut, (p.g.seg_begin + s) * p.g.seg_rows + mi * 256};
     }
     __device__ static int num_kb(const Params& p, const Tile&) { return (p.d + kBK - 1) / kBK; }
     __device__ static void prefetch(const Params& p) { FwdHidden<ACT>::prefetch(p); }
     __device__ static void load(const Params& p, const Tile& ti, int kb, uint32_t rank, uint32_t st,
                                 uint32_t bar) {
         const int k0 = kb * kBK;
-        tma_load_2d_pair(st, &p.tmX, bar, k0,
-                         (p.g.seg_begin + ti.s) * p.g.seg_rows + ti.mi * 256 + rank * 128);
-        const int c = p.g.shard_col(ti.s) + ti.nj * kOut;
+        tma_load_2d_pair(st, &p.tmX, bar, k0, ti.xrow + static_cast<int>(rank) * 128);
+        const int c = ti.c;
         if (ACT == 1) {
             const CUtensorMap* w = rank == 0 ? &p.tmG : &p.tmU;
             tma_load_2d_pair(st + kABytes, w, bar, c, k0);
@@ -268,6 +276,10 @@ struct DownAccumPair {
     static constexpr uint32_t kIdesc = make_idesc_bf16(256, BN, false, B_MN);
     struct Tile {
         int s, mi, nj;
+        int kbase;  // hidden unit of the K loop's first column (shard base, or the
+                    // ring start (seg_begin + s) fs with rot_P)
+        int kwrap;  // rot_P fs: the K loop's hidden units wrap at this column
+        int arow;   // first A row of the pair's 256 rows
     };
     __host__ __device__ static int pair_mtiles(const SegGeom& g) { return (g.seg_rows + 255) >> 8; }
     __host__ __device__ static int ntiles_n(const Params& p) { return (p.n_out + BN - 1) / BN; }
@@ -277,7 +289,12 @@ struct DownAccumPair {
     __device__ static Tile tile(const Params& p, int t) {
         const int mt = pair_mtiles(p.g), per_seg = mt * ntiles_n(p);
         const int s = t / per_seg, r = t - s * per_seg;
-        return Tile{s, r % mt, r / mt};
+        const int nj = r / mt;
+        const int mi = r - nj * mt;
+        // everything the per-k-block loads need, computed once a tile
+        return Tile{s, mi, nj,
+                    p.rot_P > 0 ? (p.g.seg_begin + s) * p.g.fs : p.g.shard_col(s),
+                    p.rot_P * p.g.fs, s * p.g.seg_rows + mi * 256};
     }
     __device__ static int num_kb(const Params& p, const Tile&) {
         return NSEG * ((p.kdim + kBK - 1) / kBK);
@@ -294,18 +311,15 @@ struct DownAccumPair {
         const CUtensorMap* ta = seg ? &p.tmA1 : &p.tmA0;
         const CUtensorMap* tb = seg ? &p.tmB1 : &p.tmB0;
         // hidden column of this k-block in H (ka) and in the weights (kw)
-        int ka = k, kw = p.g.shard_col(ti.s) + k;
+        int ka = k, kw = ti.kbase + k;
         if (p.rot_P > 0) {
             // H holds every hidden unit; segment s visits the shards in ring
             // order, starting at shard seg_begin + s (< P): column k of the
             // loop is hidden unit (k + (seg_begin + s) fs) mod (P fs).  No
             // division: this runs once per k-block in the producer thread.
-            const int f_all = p.rot_P * p.g.fs;
-            ka = k + (p.g.seg_begin + ti.s) * p.g.fs;
-            if (ka >= f_all) ka -= f_all;
-            kw = ka;
+            ka = kw = kw >= ti.kwrap ? kw - ti.kwrap : kw;
         }
-        tma_load_2d_pair(st, ta, bar, ka, ti.s * p.g.seg_rows + ti.mi * 256 + rank * 128);
+        tma_load_2d_pair(st, ta, bar, ka, ti.arow + static_cast<int>(rank) * 128);
         const int n0 = ti.nj * BN + static_cast<int>(rank) * kHalf;
         if (B_MN) {
 #pragma unroll
