@@ -49,6 +49,10 @@ def gpu_backward(inp, P, act, ws_bytes=None):
 
 
 CASES = [
+    # degenerate: one token, d_model = 8, 8-column shards
+    ("swiglu", 1, 8, 8, 1),
+    ("swiglu", 3, 16, 64, 8),
+    ("gelu", 257, 8, 16, 2),
     ("swiglu", 128, 64, 128, 1),
     ("swiglu", 256, 256, 512, 2),
     ("swiglu", 1000, 520, 1408, 8),

@@ -113,6 +113,45 @@ BF16_CASES = [
 ]
 
 
+# Degenerate shapes: one token, the narrowest rows TMA takes (d_model = 8),
+# 8-column shards, odd P -- every tile mostly zero-filled padding.
+DEGENERATE_CASES = [
+    ("swiglu", 1, 8, 8, 1),
+    ("swiglu", 3, 16, 64, 8),
+    ("gelu", 257, 8, 16, 2),
+    ("swiglu", 513, 24, 40, 5),
+]
+
+
+@pytest.mark.parametrize("act,n,d,f,P", DEGENERATE_CASES)
+def test_bf16_degenerate_shapes(act, n, d, f, P):
+    wl = small(act, "bf16", n, d, f, P, seed=31)
+    inp = make_inputs(wl)
+    Y = gpu_forward(inp, P, act)
+    ref = oracle.mlp_forward(inp["X"], inp["A"], inp["Wu"], inp["B"], act)
+    check(Y, ref, "bf16", wl.name)
+
+
+@pytest.mark.parametrize("n,d,f,P", [(8, 8, 8 * 8, 8), (16, 16, 2 * 64, 2)])
+def test_bf16_tsp_ring_degenerate(n, d, f, P):
+    """One-token and eight-token sequence shards (per-step ring passes with
+    8-column shards; rotated passes with 64-column shards)."""
+    wl = small("swiglu", "bf16", n, d, f, P, seed=32)
+    inp = make_inputs(wl)
+    Y = gpu_forward(inp, P, "swiglu", "tsp_ring")
+    ref = oracle.mlp_tsp(inp["X"], inp["A"], inp["Wu"], inp["B"], "swiglu", P)
+    check(Y, ref, "bf16", "tsp ring degenerate")
+
+
+@pytest.mark.parametrize("act,n,d,f,P", [("gelu", 1, 1, 1, 1), ("swiglu", 5, 3, 6, 3)])
+def test_fp32_degenerate_shapes(act, n, d, f, P):
+    wl = small(act, "f32", n, d, f, P, seed=33, w_std=0.3)
+    inp = make_inputs(wl)
+    Y = gpu_forward(inp, P, act)
+    ref = oracle.mlp_forward(inp["X"], inp["A"], inp["Wu"], inp["B"], act)
+    check(Y, ref, "f32", wl.name)
+
+
 @pytest.mark.parametrize("sched", ["weight_shards", "shard_passes_fused", "fused"])
 @pytest.mark.parametrize("act,n,d,f,P", BF16_CASES)
 def test_bf16_small_shapes(act, n, d, f, P, sched):
