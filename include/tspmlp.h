@@ -139,12 +139,13 @@ TSP_API tsp_status_t tsp_mlp_forward(const void* X, const void* W_gate, const vo
  *              ones bf16; TSP_SCHED_TSP_RING_FUSED also (d_ff / P) % 64 == 0)
  *   workspace  256-byte aligned device buffer, not overlapping any argument.
  *              tsp_mlp_workspace_size() gives the preferred size.  For bf16 a
- *              smaller workspace is accepted: the schedule then uses narrower
- *              hidden chunks (or fewer sequence shards per ring launch), i.e.
- *              more passes over the fp32 accumulator, down to one 128-column
- *              chunk (one sequence shard) plus the [n][d_model] fp32
- *              accumulator; below that the call returns TSP_ERR_WORKSPACE.
- *              fp32 needs the preferred size.
+ *              smaller workspace is accepted: the schedule then runs fewer
+ *              token rows (or sequence shards) a launch while 256 rows of all
+ *              d_ff hidden units still fit, and below that narrower hidden
+ *              chunks whose partial outputs go through an [n][d_model] fp32
+ *              accumulator, down to one 128-column chunk (one sequence shard)
+ *              plus that accumulator; below that the call returns
+ *              TSP_ERR_WORKSPACE.  fp32 needs the preferred size.
  * Other arguments as tsp_mlp_forward. */
 TSP_API tsp_status_t tsp_mlp_forward_ex(const void* X, const void* W_gate, const void* W_up,
                                 const void* W_down, int64_t n_tokens, int64_t d_model,
