@@ -90,7 +90,7 @@ typedef enum {
     /* Folded tensor-and-sequence ring: tokens form P equal sequence shards;
      * at ring step t sequence shard s meets weight shard (s + t) mod P, and
      * each sequence shard sums its partial outputs in that ring order.  Needs
-     * n % P == 0.  bf16 with (d_ff / P) % 64 == 0: per group of sequence
+     * n % P == 0.  bf16 with (d_ff / P) % 128 == 0: per group of sequence
      * shards (as many as fit 512 MB of hidden activations) one gate/up launch
      * over all d_ff columns and one down projection whose K loop runs over
      * the weight shards in each sequence shard's ring order, summing in

@@ -18,6 +18,7 @@ struct WgradPair {
     using Base = Wgrad<NCOLS, SPLIT>;
     using Params = typename Base::Params;
     static constexpr const char* kName = Base::kName;
+    // 64-deep k-blocks (tokens): 128-deep ones measured the same within noise
     static constexpr int kBK = 64;
     static constexpr int kABytes = 128 * kBK * 2;
     static constexpr int kStageBytes = kABytes + (NCOLS / 2) * kBK * 2;
@@ -64,6 +65,7 @@ struct WgradPair {
     __device__ static void mma(const Tile&, int kb, uint32_t st, uint32_t acc) {
 #pragma unroll
         for (int kk = 0; kk < kBK / 16; ++kk) {
+            // MN-major: 2 KB a K16 step; the next 64-column box 8 KB on
             const uint64_t a = make_smem_desc(st + 2048 * kk, 8192, 1024, kLayoutSW128);
             const uint64_t b = make_smem_desc(st + kABytes + 2048 * kk, 8192, 1024, kLayoutSW128);
             umma_bf16_pair(acc, a, b, kIdesc, (kb | kk) != 0 ? 1u : 0u);
@@ -100,6 +102,7 @@ template <int ACT>
 struct DhPair {
     using Params = DhParams;
     static constexpr const char* kName = ACT == 1 ? "bwd_dh_swiglu" : "bwd_dh_gelu";
+    // 64-deep k-blocks: 128-deep ones measured the same within noise
     static constexpr int kBK = 64;
     static constexpr int kABytes = 128 * kBK * 2;
     static constexpr int kStageBytes = kABytes + 128 * kBK * 2;
@@ -169,11 +172,12 @@ template <int ACT>
 struct BwdGateUpPair {
     using Params = BwdGateUpParams;
     static constexpr const char* kName = ACT == 1 ? "bwd_gate_up_swiglu" : "bwd_gate_up_gelu";
-    static constexpr int kBK = 64;
+    // 128-deep k-blocks as FwdHiddenPair
+    static constexpr int kBK = 128;
     static constexpr int kOut = ACT == 1 ? 128 : 256;
     static constexpr int kABytes = 128 * kBK * 2;
     static constexpr int kStageBytes = kABytes + 128 * kBK * 2;
-    static constexpr int kStages = 6;
+    static constexpr int kStages = 3;
     static constexpr int kAccCols = 256, kAccBufs = 2;
     static constexpr uint32_t kIdesc = make_idesc_bf16(256, 256, false, true);
     struct Tile {
@@ -195,23 +199,26 @@ struct BwdGateUpPair {
     __device__ static void load(const Params& p, const Tile& ti, int kb, uint32_t rank, uint32_t st,
                                 uint32_t bar) {
         const int k0 = kb * kBK;
-        tma_load_2d_pair(st, &p.tmX, bar, k0, ti.mi * 256 + static_cast<int>(rank) * 128);
+        const int xr = ti.mi * 256 + static_cast<int>(rank) * 128;
+        tma_load_2d_pair(st, &p.tmX, bar, k0, xr);
+        tma_load_2d_pair(st + 16384, &p.tmX, bar, k0 + 64, xr);
         const int c = p.col_base + ti.nj * kOut;
         if (ACT == 1) {
             const CUtensorMap* w = rank == 0 ? &p.tmG : &p.tmU;
             tma_load_2d_pair(st + kABytes, w, bar, c, k0);
-            tma_load_2d_pair(st + kABytes + 8192, w, bar, c + 64, k0);
+            tma_load_2d_pair(st + kABytes + 16384, w, bar, c + 64, k0);
         } else {
             const int cr = c + static_cast<int>(rank) * 128;
             tma_load_2d_pair(st + kABytes, &p.tmG, bar, cr, k0);
-            tma_load_2d_pair(st + kABytes + 8192, &p.tmG, bar, cr + 64, k0);
+            tma_load_2d_pair(st + kABytes + 16384, &p.tmG, bar, cr + 64, k0);
         }
     }
     __device__ static void mma(const Tile&, int kb, uint32_t st, uint32_t acc) {
 #pragma unroll
         for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t a = make_smem_desc(st + 32 * kk, 16, 1024, kLayoutSW128);
-            const uint64_t b = make_smem_desc(st + kABytes + 2048 * kk, 8192, 1024, kLayoutSW128);
+            const uint64_t a =
+                make_smem_desc(st + (kk >> 2) * 16384 + 32 * (kk & 3), 16, 1024, kLayoutSW128);
+            const uint64_t b = make_smem_desc(st + kABytes + 2048 * kk, 16384, 1024, kLayoutSW128);
             umma_bf16_pair(acc, a, b, kIdesc, (kb | kk) != 0 ? 1u : 0u);
         }
     }

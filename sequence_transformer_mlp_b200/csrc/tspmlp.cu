@@ -434,7 +434,7 @@ FwdPlan plan_forward_budget(int64_t n, int64_t d, int64_t f, int P, tsp_dtype_t 
         // its ring order (no fp32 accumulator), for as many sequence shards a
         // launch as fit the budget
         const size_t per_seg_all = static_cast<size_t>(n / P) * f * e;
-        if (dt == TSP_DT_BF16 && fs % 64 == 0 && budget >= per_seg_all) {
+        if (dt == TSP_DT_BF16 && fs % 128 == 0 && budget >= per_seg_all) {
             pl.ring_rotated = true;
             pl.tsp_group = static_cast<int>(
                 std::min<size_t>(P, std::max<size_t>(1, std::min(budget, kRingGroupBudget) / per_seg_all)));
@@ -590,8 +590,8 @@ tsp_status_t fwd_pass_bf16(const void* X, const void* Wg, const void* Wu, const 
     typename K1::Params p1;
     std::memset(&p1, 0, sizeof(p1));
     if (!tmap_bf16(&p1.tmX, X, d, n, d, 64, 128, SW128) ||
-        !tmap_bf16(&p1.tmG, Wg, f, d, f, 64, 64, SW128) ||
-        (ACT == 1 && !tmap_bf16(&p1.tmU, Wu, f, d, f, 64, 64, SW128)))
+        !tmap_bf16(&p1.tmG, Wg, f, d, f, 64, 128, SW128) ||
+        (ACT == 1 && !tmap_bf16(&p1.tmU, Wu, f, d, f, 64, 128, SW128)))
         return TSP_ERR_CUDA;
     p1.g = g;
     p1.d = static_cast<int>(d);
@@ -604,7 +604,7 @@ tsp_status_t fwd_pass_bf16(const void* X, const void* Wg, const void* Wu, const 
     std::memset(&p2, 0, sizeof(p2));
     const int64_t hrows = static_cast<int64_t>(g.num_segs) * g.seg_rows;
     if (!tmap_bf16(&p2.tmA0, H, width, hrows, width, 64, 128, SW128) ||
-        !tmap_bf16(&p2.tmB0, Wd, d, f, d, 64, 64, SW128))
+        !tmap_bf16(&p2.tmB0, Wd, d, f, d, 64, 128, SW128))
         return TSP_ERR_CUDA;
     p2.g = g;
     p2.kdim = static_cast<int>(width);
@@ -966,8 +966,8 @@ tsp_status_t backward_bf16(const void* X, const void* Wg, const void* Wu, const 
             BwdGateUpParams p;
             std::memset(&p, 0, sizeof(p));
             if (!tmap_bf16(&p.tmX, X, d, n, d, 64, 128, SW128) ||
-                !tmap_bf16(&p.tmG, Wg, f, d, f, 64, 64, SW128) ||
-                (ACT == 1 && !tmap_bf16(&p.tmU, Wu, f, d, f, 64, 64, SW128)))
+                !tmap_bf16(&p.tmG, Wg, f, d, f, 64, 128, SW128) ||
+                (ACT == 1 && !tmap_bf16(&p.tmU, Wu, f, d, f, 64, 128, SW128)))
                 return TSP_ERR_CUDA;
             p.n = static_cast<int>(n);
             p.d = static_cast<int>(d);
