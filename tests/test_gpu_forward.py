@@ -310,7 +310,8 @@ def llama8b():
     return _full_inputs(LLAMA8B)
 
 
-@pytest.mark.parametrize("P,sched", [(8, "weight_shards"), (4, "weight_shards"),
+@pytest.mark.parametrize("P,sched", [(8, "weight_shards"), (7, "weight_shards"),
+                                     (4, "weight_shards"),
                                      (2, "weight_shards"), (1, "weight_shards"),
                                      (8, "shard_passes_fused"), (8, "fused"), (1, "fused")])
 def test_llama8b_shape_sampled_rows(llama8b, P, sched):
