@@ -424,7 +424,9 @@ __global__ void __launch_bounds__(kPipelineThreads, 1)
                                 a4[i] = o;
                             }
                         } else {
-                            for (int i = 0; i < valid; ++i) a[i] += __uint_as_float(v[i]);
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                if (i < valid) a[i] += __uint_as_float(v[i]);
                         }
                     } else {
                         uint32_t pk[16];

@@ -59,9 +59,13 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const uint32_t
         for (int i = 0; i < 4; ++i)
             d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
     } else {
+        // unrolled with constant indices, so pk stays in registers (a
+        // run-time index would put it on the stack for every call)
         uint16_t* d16 = reinterpret_cast<uint16_t*>(dst);
-        for (int i = 0; i < valid; ++i)
-            d16[i] = static_cast<uint16_t>((i & 1) ? (pk[i >> 1] >> 16) : (pk[i >> 1] & 0xFFFFu));
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            if (i < valid)
+                d16[i] = static_cast<uint16_t>((i & 1) ? (pk[i >> 1] >> 16) : (pk[i >> 1] & 0xFFFFu));
     }
 }
 
@@ -73,7 +77,9 @@ __device__ __forceinline__ void store_f32x32(float* dst, const uint32_t (&v)[32]
             d4[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
                                 __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
     } else {
-        for (int i = 0; i < valid; ++i) dst[i] = __uint_as_float(v[i]);
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            if (i < valid) dst[i] = __uint_as_float(v[i]);
     }
 }
 
@@ -255,7 +261,9 @@ struct DownAccum {
                         a4[i] = o;
                     }
                 } else {
-                    for (int i = 0; i < valid; ++i) a[i] += __uint_as_float(v[i]);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (i < valid) a[i] += __uint_as_float(v[i]);
                 }
             } else {
                 uint32_t pk[16];
