@@ -49,6 +49,8 @@ FORWARD_SOURCES = ["ptx.cuh", "pipeline.cuh", "pipeline2.cuh", "recipes.cuh"]
 
 
 def kernel_sources(kernel: str) -> list[str]:
+    if kernel.endswith("_save") or kernel.startswith("bwd_dh_factor"):
+        return FORWARD_SOURCES + ["bwd_pair.cuh", "train_pair.cuh"]
     if kernel.startswith("fused_fwd"):
         return FORWARD_SOURCES + ["fused.cuh"]
     if kernel.startswith("fused_passes"):
@@ -305,6 +307,10 @@ def main():
                     help="override the workload's schedule")
     ap.add_argument("--P", type=int, default=None,
                     help="override the workload's number of logical weight shards")
+    ap.add_argument("--bwd-recompute", action="store_true",
+                    help="fwd+bwd workloads: the inference forward and the backward that "
+                         "recomputes the gate/up projection, instead of the training forward "
+                         "that keeps its activations")
     ap.add_argument("--ref-rows", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true",
@@ -346,17 +352,34 @@ def main():
     dt = "f32" if wl.dtype == "f32" else "bf16"
     tdt = torch.float32 if dt == "f32" else torch.bfloat16
     Y = torch.empty(n, d, dtype=tdt, device="cuda")
-    need = T.tsp_mlp_workspace_size(n, d, f, P, wl.act, dt, sched, backward=wl.backward)
+    saved_act = wl.backward and not args.bwd_recompute
+    if not wl.backward:
+        need = T.tsp_mlp_workspace_size(n, d, f, P, wl.act, dt, sched)
+    elif saved_act:
+        need = T.tsp_mlp_backward_saved_workspace_size(n, d, f, P, wl.act)
+    else:
+        need = T.tsp_mlp_workspace_size(n, d, f, P, wl.act, dt, sched, backward=True)
     ws = torch.empty(max(need, 1), dtype=torch.uint8, device="cuda")
     if wl.backward:
         dX = torch.empty(n, d, dtype=torch.bfloat16, device="cuda")
         dWg = torch.empty(d, f, dtype=torch.float32, device="cuda")
-        dWu = torch.empty(d, f, dtype=torch.float32, device="cuda")
+        dWu = torch.empty(d, f, dtype=torch.float32, device="cuda") if wl.act == "swiglu" else None
         dWd = torch.empty(f, d, dtype=torch.float32, device="cuda")
-        ws_f = torch.empty(max(T.tsp_mlp_workspace_size(n, d, f, P, wl.act, "bf16", sched), 1),
-                           dtype=torch.uint8, device="cuda")
+        if saved_act:
+            # the training forward keeps H and the activation's factors for the backward
+            n_saved = T.tsp_mlp_saved_size(n, d, f, P, wl.act)
+            saved = torch.empty(n_saved, dtype=torch.uint8, device="cuda")
+        else:
+            ws_f = torch.empty(max(T.tsp_mlp_workspace_size(n, d, f, P, wl.act, "bf16", sched), 1),
+                               dtype=torch.uint8, device="cuda")
 
     def step(x=dev["X"], y=Y):
+        if saved_act:
+            T.tsp_mlp_forward_train(x, dev["A"], dev["Wu"], dev["B"], n, d, f, P, wl.act, y, saved,
+                                    n_saved, stream)
+            T.tsp_mlp_backward_saved(x, dev["A"], dev["Wu"], dev["B"], dev["dY"], saved, n_saved,
+                                     n, d, f, P, wl.act, dX, dWg, dWu, dWd, ws, need, stream)
+            return
         T.tsp_mlp_forward_ex(x, dev["A"], dev["Wu"], dev["B"], n, d, f, P, wl.act, dt, sched,
                              y, ws_f if wl.backward else ws,
                              ws_f.numel() if wl.backward else need, stream)
@@ -431,6 +454,8 @@ def main():
             "pct_of_bf16_peak_sustained": 100.0 * tflops / (world * pk["bf16_tflops_sustained"]),
             "config": {"workload": wl.name, "n_tokens": n, "d_model": d, "d_ff": f, "P": P,
                        "act": wl.act, "schedule": sched, "parallelism": f"replicas{world}",
+                       **({"backward": "saved activations" if saved_act else "recompute"}
+                          if wl.backward else {}),
                        "l2": "inputs larger than L2 (weights 3 x d x f bf16), no flush"
                        if dt == "bf16" else "inputs fit in L2 (launch-latency bound), no flush"},
             "roofline": {"bound": bound, "kernel": dom, "achieved": achieved,
@@ -472,14 +497,19 @@ def kernel_flops_per_step(kernel: str, wl) -> float:
     product it computes).  Per step the forward hidden kernel covers all n x f
     hidden units once and the down kernel all n x d outputs over K = d_ff,
     whatever the number of launches (chunks, ring steps) they are split into.
-    The backward's recomputed gate/up products are counted: they run on the
-    tensor cores like the rest."""
+    The recompute backward's gate/up products are counted too: they run on the
+    tensor cores like the rest (the fwd+bwd step's default path, the training
+    forward that keeps its activations, has none)."""
     n, d, f = wl.n, wl.d, wl.f
     return {
         "fused_fwd_swiglu": 2 * 3 * n * d * f,
         "fused_fwd_gelu": 2 * 2 * n * d * f,
         "fwd_hidden_swiglu": 2 * 2 * n * d * f,
         "fwd_hidden_gelu": 2 * n * d * f,
+        "fwd_hidden_swiglu_save": 2 * 2 * n * d * f,
+        "fwd_hidden_gelu_save": 2 * n * d * f,
+        "bwd_dh_factor_swiglu": 2 * n * d * f,
+        "bwd_dh_factor_gelu": 2 * n * d * f,
         "down_accum_fwd": 2 * n * d * f,
         "fused_passes_swiglu": 2 * 3 * n * d * f,
         "fused_passes_gelu": 2 * 2 * n * d * f,

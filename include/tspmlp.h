@@ -211,6 +211,60 @@ TSP_API tsp_status_t tsp_mlp_workspace_size(int64_t n_tokens, int64_t d_model, i
                                     tsp_act_t act, tsp_dtype_t dtype, tsp_sched_t sched,
                                     int backward, size_t* bytes);
 
+/* Training: a forward that keeps its activations, and a backward that uses
+ * them instead of recomputing the gate/up projection from X.
+ *
+ * The backward of the block needs, at every hidden unit, dH = dY.W_down^T
+ * times the derivative of the activation ("Folding Tensor and Sequence
+ * Parallelism ...", Abstract: the gated form; "Tensor Parallelism: Splitting
+ * the Math": the plain block).  tsp_mlp_forward_train writes, besides Y, the
+ * activations and the activation's derivative factors at every hidden unit:
+ *   H  = h(X)                    bf16 [n_tokens][d_ff]  (as the forward's)
+ *   S1 = SiLU(G)  (SwiGLU)  or  GeLU'(Z) (GeLU)          fp32 [n_tokens][d_ff]
+ *   S2 = U SiLU'(G)  (SwiGLU only)                       fp32 [n_tokens][d_ff]
+ * with G = X.W_gate, U = X.W_up, Z = X.A, SiLU'(g) = s (1 + g (1 - s)),
+ * s = sigmoid(g), GeLU'(z) = Phi(z) + z phi(z); and tsp_mlp_backward_saved
+ * forms dU = dH S1 and dG = dH S2 (GeLU: dG = dH S1) in the epilogue of the
+ * dH product, so dH is never stored.  The factors are evaluated exactly as
+ * tsp_mlp_backward_ex evaluates them from its recomputed G and U, so dX,
+ * dW_gate and dW_up are bit-identical to its results; dW_down uses the
+ * forward's H.
+ *
+ * The saved buffer is opaque to the caller: H, then S1, then S2, each region
+ * 256-byte aligned; tsp_mlp_saved_size gives its size.  It must be 256-byte
+ * aligned and overlap no other argument; the backward only reads it. */
+TSP_API tsp_status_t tsp_mlp_saved_size(int64_t n_tokens, int64_t d_model, int64_t d_ff, int P,
+                                        tsp_act_t act, size_t* bytes);
+
+/* Forward pass (bf16, weight-shard schedule) that also fills `saved`.  Y as
+ * tsp_mlp_forward (bit-identical to it); requirements as tsp_mlp_forward.  H
+ * lives in `saved`, so no workspace is needed: token rows run in groups of
+ * at most 128 MB of H (as the pass schedule's row groups), each one gate/up
+ * launch writing H, S1 (S2) and one down projection reading H. */
+TSP_API tsp_status_t tsp_mlp_forward_train(const void* X, const void* W_gate, const void* W_up,
+                                           const void* W_down, int64_t n_tokens, int64_t d_model,
+                                           int64_t d_ff, int P, tsp_act_t act, void* Y,
+                                           void* saved, size_t saved_bytes, tsp_stream_t stream);
+
+/* Preferred workspace bytes of tsp_mlp_backward_saved: the dG (dU) chunk
+ * buffers and, with more than one chunk, the fp32 dX accumulator. */
+TSP_API tsp_status_t tsp_mlp_backward_saved_workspace_size(int64_t n_tokens, int64_t d_model,
+                                                           int64_t d_ff, int P, tsp_act_t act,
+                                                           size_t* bytes);
+
+/* Backward pass from the activations tsp_mlp_forward_train saved for the
+ * same X and weights.  Outputs, requirements and the smaller-workspace rule
+ * as tsp_mlp_backward_ex.  Per hidden chunk: the dH product with the factors
+ * applied (dG, dU to the workspace), dW_down = H^T.dY from the saved H,
+ * dW_gate (dW_up) = X^T.dG (dU), and dX (+)= dG.W_gate^T (+ dU.W_up^T). */
+TSP_API tsp_status_t tsp_mlp_backward_saved(const void* X, const void* W_gate, const void* W_up,
+                                            const void* W_down, const void* dY, const void* saved,
+                                            size_t saved_bytes, int64_t n_tokens, int64_t d_model,
+                                            int64_t d_ff, int P, tsp_act_t act, void* dX,
+                                            float* dW_gate, float* dW_up, float* dW_down,
+                                            void* workspace, size_t workspace_bytes,
+                                            tsp_stream_t stream);
+
 /* A static, human-readable name for a status. */
 TSP_API const char* tsp_status_string(tsp_status_t status);
 

@@ -74,6 +74,12 @@ def load(path: str | None = None) -> ctypes.CDLL:
                                         vp, vp, sz, vp]
     lib.tsp_mlp_workspace_size.argtypes = [i64, i64, i64, ci, ci, ci, ci, ci,
                                            ctypes.POINTER(ctypes.c_size_t)]
+    lib.tsp_mlp_saved_size.argtypes = [i64, i64, i64, ci, ci, ctypes.POINTER(ctypes.c_size_t)]
+    lib.tsp_mlp_forward_train.argtypes = [vp, vp, vp, vp, i64, i64, i64, ci, ci, vp, vp, sz, vp]
+    lib.tsp_mlp_backward_saved_workspace_size.argtypes = [i64, i64, i64, ci, ci,
+                                                          ctypes.POINTER(ctypes.c_size_t)]
+    lib.tsp_mlp_backward_saved.argtypes = [vp, vp, vp, vp, vp, vp, sz, i64, i64, i64, ci, ci, vp,
+                                           vp, vp, vp, vp, sz, vp]
     lib.tsp_status_string.argtypes = [ci]
     lib.tsp_status_string.restype = ctypes.c_char_p
     lib.tsp_poll_device_error.argtypes = [vp]
@@ -85,7 +91,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
                  "tsp_mlp_backward",
                  "tsp_mlp_backward_ex", "tsp_mlp_workspace_size", "tsp_poll_device_error",
                  "tsp_trace_enable", "tsp_trace_collect", "tsp_trace_reset",
-                 "tsp_selftest_timeout"):
+                 "tsp_selftest_timeout", "tsp_mlp_saved_size", "tsp_mlp_forward_train",
+                 "tsp_mlp_backward_saved_workspace_size", "tsp_mlp_backward_saved"):
         getattr(lib, name).restype = ci
     if path is None:
         _lib = lib
@@ -183,6 +190,44 @@ def tsp_mlp_workspace_size(n_tokens, d_model, d_ff, P, act, dtype="bf16", sched=
                                       1 if backward else 0, ctypes.byref(out))
     _check(s, "tsp_mlp_workspace_size")
     return int(out.value)
+
+
+def tsp_mlp_saved_size(n_tokens, d_model, d_ff, P, act) -> int:
+    out = ctypes.c_size_t(0)
+    s = load().tsp_mlp_saved_size(n_tokens, d_model, d_ff, P, _enum(ACT, act), ctypes.byref(out))
+    _check(s, "tsp_mlp_saved_size")
+    return int(out.value)
+
+
+def tsp_mlp_forward_train(X, W_gate, W_up, W_down, n_tokens, d_model, d_ff, P, act, Y, saved,
+                          saved_bytes, stream=None, check=True) -> int:
+    s = load().tsp_mlp_forward_train(_addr(X), _addr(W_gate), _addr(W_up), _addr(W_down),
+                                     n_tokens, d_model, d_ff, P, _enum(ACT, act), _addr(Y),
+                                     _addr(saved), saved_bytes, _stream(stream))
+    if check:
+        _check(s, "tsp_mlp_forward_train")
+    return s
+
+
+def tsp_mlp_backward_saved_workspace_size(n_tokens, d_model, d_ff, P, act) -> int:
+    out = ctypes.c_size_t(0)
+    s = load().tsp_mlp_backward_saved_workspace_size(n_tokens, d_model, d_ff, P, _enum(ACT, act),
+                                                     ctypes.byref(out))
+    _check(s, "tsp_mlp_backward_saved_workspace_size")
+    return int(out.value)
+
+
+def tsp_mlp_backward_saved(X, W_gate, W_up, W_down, dY, saved, saved_bytes, n_tokens, d_model,
+                           d_ff, P, act, dX, dW_gate, dW_up, dW_down, workspace, workspace_bytes,
+                           stream=None, check=True) -> int:
+    s = load().tsp_mlp_backward_saved(_addr(X), _addr(W_gate), _addr(W_up), _addr(W_down),
+                                      _addr(dY), _addr(saved), saved_bytes, n_tokens, d_model,
+                                      d_ff, P, _enum(ACT, act), _addr(dX), _addr(dW_gate),
+                                      _addr(dW_up), _addr(dW_down), _addr(workspace),
+                                      workspace_bytes, _stream(stream))
+    if check:
+        _check(s, "tsp_mlp_backward_saved")
+    return s
 
 
 def tsp_status_string(status: int) -> str:

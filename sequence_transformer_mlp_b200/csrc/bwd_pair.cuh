@@ -8,6 +8,27 @@
 
 namespace tspmlp {
 
+// Derivative factors of the activations, with every rounding written out (no
+// multiply-add left for the compiler to fuse or not), so that the recompute
+// backward here and the training forward (train_pair.cuh) get the same bits.
+//   sigmoid(g) = 1 / (1 + exp(-g))
+//   SiLU'(g) u = u s (1 + g (1 - s)),  s = sigmoid(g)
+//   GeLU'(z)   = Phi(z) + z phi(z),  Phi(z) = (1 + erf(z / sqrt 2)) / 2,
+//                phi(z) = exp(-z^2 / 2) / sqrt(2 pi)
+__device__ __forceinline__ float sigmoid_rn(float g) {
+    return __fdiv_rn(1.0f, __fadd_rn(1.0f, __expf(-g)));
+}
+__device__ __forceinline__ float swiglu_gate_factor(float g, float u, float s) {
+    return __fmul_rn(__fmul_rn(u, s), __fmaf_rn(g, __fsub_rn(1.0f, s), 1.0f));
+}
+__device__ __forceinline__ float gelu_cdf_rn(float z) {
+    return __fmul_rn(0.5f, __fadd_rn(1.0f, erff(__fmul_rn(z, 0.70710678118654752440f))));
+}
+__device__ __forceinline__ float gelu_grad_rn(float z, float cdf) {
+    const float pdf = __fmul_rn(0.39894228040143267794f, __expf(__fmul_rn(__fmul_rn(-0.5f, z), z)));
+    return __fmaf_rn(z, pdf, cdf);
+}
+
 // ============================================================================
 // Paired weight gradients (see Wgrad): both operands MN-major, K = tokens.
 // Tile = 256 output rows x NCOLS output columns; CTA r stages 128 of the rows
@@ -88,7 +109,7 @@ struct WgradPair {
 //   SwiGLU: H = SiLU(G) U,  dU = dH SiLU(G),  dG = dH U SiLU'(G)   (bf16)
 //   GeLU:   H = GeLU(G),    dG = dH GeLU'(G)                        (bf16)
 // with SiLU'(g) = s (1 + g (1 - s)), s = sigmoid(g), and GeLU'(z) = Phi(z) +
-// z phi(z): the derivatives of the forward definition.  dH stays fp32, so
+// z phi(z): the derivatives of the forward definition (helpers above).  dH stays fp32, so
 // the only roundings are those of H, dG and dU to bf16.
 struct DhParams {
     CUtensorMap tmDY;  // dY [n][d], box {64, 128}
@@ -265,11 +286,11 @@ struct BwdGateUpPair {
 #pragma unroll
                     for (int j = 0; j < 2; ++j) {
                         const float gv = __uint_as_float(g[2 * i + j]), uv = __uint_as_float(u[2 * i + j]);
-                        const float sg = 1.0f / (1.0f + __expf(-gv));
-                        const float si = gv * sg;
+                        const float sg = sigmoid_rn(gv);
+                        const float si = __fmul_rn(gv, sg);
                         h[j] = si * uv;
                         duv[j] = dh[2 * i + j] * si;
-                        dgv[j] = dh[2 * i + j] * (uv * sg * (1.0f + gv * (1.0f - sg)));
+                        dgv[j] = dh[2 * i + j] * swiglu_gate_factor(gv, uv, sg);
                     }
                     ph[i] = pack_bf16x2(h[0], h[1]);
                     pg[i] = pack_bf16x2(dgv[0], dgv[1]);
@@ -285,10 +306,9 @@ struct BwdGateUpPair {
 #pragma unroll
                     for (int j = 0; j < 2; ++j) {
                         const float z = __uint_as_float(g[2 * i + j]);
-                        const float cdf = 0.5f * (1.0f + erff(z * 0.70710678118654752440f));
-                        const float pdf = 0.39894228040143267794f * __expf(-0.5f * z * z);
+                        const float cdf = gelu_cdf_rn(z);
                         h[j] = z * cdf;
-                        dgv[j] = dh[2 * i + j] * (cdf + z * pdf);
+                        dgv[j] = dh[2 * i + j] * gelu_grad_rn(z, cdf);
                     }
                     ph[i] = pack_bf16x2(h[0], h[1]);
                     pg[i] = pack_bf16x2(dgv[0], dgv[1]);

@@ -1,0 +1,162 @@
+// train_pair.cuh -- the training forward that keeps what the backward needs,
+// and the backward's first GEMM that reads it.
+//
+// The recompute backward (bwd_pair.cuh) runs the gate/up projection a second
+// time to get G and U back.  Here the forward's gate/up epilogue, which has G
+// and U in tensor memory anyway, also writes the activation's derivative
+// factors in fp32, and the dH GEMM's epilogue turns dH into dG (and dU) with
+// them directly:
+//   SwiGLU: S1 = SiLU(G),  S2 = U SiLU'(G)   dU = dH S1,  dG = dH S2
+//   GeLU:   S1 = GeLU'(Z)                     dG = dH S1
+// with SiLU'(g) = s (1 + g (1 - s)), s = sigmoid(g), GeLU'(z) = Phi(z) +
+// z phi(z) -- the derivatives of the forward definition, evaluated by the
+// recompute backward's own helpers (bwd_pair.cuh, every rounding explicit),
+// so dG and dU come out bit for bit the same.  dH itself is never stored.
+#pragma once
+
+#include "bwd_pair.cuh"
+
+namespace tspmlp {
+
+// ============================================================================
+// Gate/up projection (as FwdHiddenPair) whose epilogue also keeps S1 (S2).
+template <int ACT>
+struct FwdHiddenSaveParams : FwdHidden<ACT>::Params {
+    float* S1;  // [rows][ldh] fp32, indexed as H
+    float* S2;  // [rows][ldh] fp32 (SwiGLU)
+};
+
+template <int ACT>
+struct FwdHiddenSavePair : FwdHiddenPair<ACT> {
+    using Base = FwdHiddenPair<ACT>;
+    using Params = FwdHiddenSaveParams<ACT>;
+    using Tile = typename Base::Tile;
+    static constexpr const char* kName = ACT == 1 ? "fwd_hidden_swiglu_save" : "fwd_hidden_gelu_save";
+
+    __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t rank, uint32_t acc,
+                                    int q, int lane) {
+        const int rl = (2 * ti.mi + static_cast<int>(rank)) * 128 + q * 32 + lane;
+        const bool row_ok = rl < p.g.seg_rows;
+        const long long off = static_cast<long long>(ti.s * p.g.seg_rows + rl) * p.ldh;
+        const uint32_t t0 = acc + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll 1
+        for (int cc = 0; cc < Base::kOut / 32; ++cc) {
+            const int c0 = ti.nj * Base::kOut + 32 * cc;
+            const int valid = p.width - c0;
+            uint32_t g[32];
+            tmem_ld_32x32b_x32(t0 + 32 * cc, g);
+            if (ACT == 1) {
+                uint32_t u[32];
+                tmem_ld_32x32b_x32(t0 + 128 + 32 * cc, u);
+                tmem_ld_wait();
+                if (!row_ok || valid <= 0) continue;
+                uint32_t pk[16], s1[32], s2[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float gv = __uint_as_float(g[i]), uv = __uint_as_float(u[i]);
+                    const float sg = sigmoid_rn(gv);
+                    s1[i] = __float_as_uint(__fmul_rn(gv, sg));
+                    s2[i] = __float_as_uint(swiglu_gate_factor(gv, uv, sg));
+                    g[i] = __float_as_uint(silu_f(gv) * uv);  // H, as the inference forward
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    pk[i] = pack_bf16x2(__uint_as_float(g[2 * i]), __uint_as_float(g[2 * i + 1]));
+                store_bf16x32(p.H + off + c0, pk, valid);
+                store_f32x32(p.S1 + off + c0, s1, valid);
+                store_f32x32(p.S2 + off + c0, s2, valid);
+            } else {
+                tmem_ld_wait();
+                if (!row_ok || valid <= 0) continue;
+                uint32_t pk[16], s1[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float z = __uint_as_float(g[i]);
+                    s1[i] = __float_as_uint(gelu_grad_rn(z, gelu_cdf_rn(z)));
+                    g[i] = __float_as_uint(gelu_f(z));
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    pk[i] = pack_bf16x2(__uint_as_float(g[2 * i]), __uint_as_float(g[2 * i + 1]));
+                store_bf16x32(p.H + off + c0, pk, valid);
+                store_f32x32(p.S1 + off + c0, s1, valid);
+            }
+        }
+    }
+};
+
+// ============================================================================
+// dH = dY . W_down[c..]^T (as DhPair), whose epilogue applies the saved
+// factors and writes dG (dU) in bf16 instead of storing dH.
+struct DhFactorParams : DhParams {
+    const float* S1;  // saved factors at the chunk's first column, row pitch lds
+    const float* S2;  // (SwiGLU)
+    long long lds;
+    __nv_bfloat16* dG;  // [n][width] at pitch ld
+    __nv_bfloat16* dU;  // [n][width] (SwiGLU)
+};
+
+template <int ACT>
+struct DhFactorPair : DhPair<ACT> {
+    using Base = DhPair<ACT>;
+    using Params = DhFactorParams;
+    using Tile = typename Base::Tile;
+    static constexpr const char* kName = ACT == 1 ? "bwd_dh_factor_swiglu" : "bwd_dh_factor_gelu";
+
+    // 32 fp32 factors from src[0..valid) (zero beyond)
+    __device__ static void load_f32x32(const float* src, int valid, float (&v)[32]) {
+        if (valid >= 32) {
+            const float4* s4 = reinterpret_cast<const float4*>(src);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float4 x = s4[i];
+                v[4 * i] = x.x;
+                v[4 * i + 1] = x.y;
+                v[4 * i + 2] = x.z;
+                v[4 * i + 3] = x.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = i < valid ? src[i] : 0.0f;
+        }
+    }
+
+    __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t rank, uint32_t acc,
+                                    int q, int lane) {
+        const int row = ti.mi * 256 + static_cast<int>(rank) * 128 + q * 32 + lane;
+        const bool row_ok = row < p.n;
+        const long long off = static_cast<long long>(row) * p.ld;
+        const long long soff = static_cast<long long>(row) * p.lds;
+        const uint32_t t0 = acc + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll 1
+        for (int cc = 0; cc < 8; ++cc) {
+            const int c0 = ti.nj * 256 + 32 * cc;
+            const int valid = p.width - c0;
+            const bool live = row_ok && valid > 0;
+            float s1[32], s2[32];
+            if (live) {
+                load_f32x32(p.S1 + soff + c0, valid, s1);
+                if (ACT == 1) load_f32x32(p.S2 + soff + c0, valid, s2);
+            }
+            uint32_t dh[32], pk[16];
+            tmem_ld_32x32b_x32(t0 + 32 * cc, dh);
+            tmem_ld_wait();
+            if (!live) continue;
+            if (ACT == 1) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    pk[i] = pack_bf16x2(__uint_as_float(dh[2 * i]) * s1[2 * i],
+                                        __uint_as_float(dh[2 * i + 1]) * s1[2 * i + 1]);
+                store_bf16x32(p.dU + off + c0, pk, valid);
+            }
+            const float(&sg)[32] = ACT == 1 ? s2 : s1;
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                pk[i] = pack_bf16x2(__uint_as_float(dh[2 * i]) * sg[2 * i],
+                                    __uint_as_float(dh[2 * i + 1]) * sg[2 * i + 1]);
+            store_bf16x32(p.dG + off + c0, pk, valid);
+        }
+    }
+};
+
+}  // namespace tspmlp

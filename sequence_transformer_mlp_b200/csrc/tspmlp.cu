@@ -20,6 +20,7 @@
 
 #include "../../include/tspmlp.h"
 #include "bwd_pair.cuh"
+#include "train_pair.cuh"
 #include "fused.cuh"
 #include "fused2.cuh"
 #include "pipeline2.cuh"
@@ -584,7 +585,8 @@ template <int ACT>
 tsp_status_t fwd_pass_bf16(const void* X, const void* Wg, const void* Wu, const void* Wd,
                            int64_t n, int64_t d, int64_t f, const SegGeom& g, int64_t width,
                            int mode, __nv_bfloat16* H, float* acc, void* Y, cudaStream_t st,
-                           int dev, int sms, int rot_P = 0) {
+                           int dev, int sms, int rot_P = 0, float* S1 = nullptr,
+                           float* S2 = nullptr) {
     using K1 = FwdHidden<ACT>;
     using K2 = DownAccum<true, 1>;
     typename K1::Params p1;
@@ -598,7 +600,17 @@ tsp_status_t fwd_pass_bf16(const void* X, const void* Wg, const void* Wu, const 
     p1.width = static_cast<int>(width);
     p1.H = H;
     p1.ldh = width;
-    TSP_TRY(launch_pair<FwdHiddenPair<ACT>>(p1, st, dev, sms));
+    if (S1) {
+        // training forward: the same tiles, keeping the activation's factors
+        FwdHiddenSaveParams<ACT> ps;
+        std::memset(&ps, 0, sizeof(ps));
+        static_cast<typename K1::Params&>(ps) = p1;
+        ps.S1 = S1;
+        ps.S2 = S2;
+        TSP_TRY(launch_pair<FwdHiddenSavePair<ACT>>(ps, st, dev, sms));
+    } else {
+        TSP_TRY(launch_pair<FwdHiddenPair<ACT>>(p1, st, dev, sms));
+    }
 
     typename K2::Params p2;
     std::memset(&p2, 0, sizeof(p2));
@@ -819,6 +831,59 @@ tsp_status_t forward_bf16(const void* X, const void* Wg, const void* Wu, const v
     return TSP_OK;
 }
 
+// ---------------------------------------------------------------------------
+// training forward: the weight-shard pass schedule with its activations kept
+
+// Saved activations: H (bf16 [n][f]), then the fp32 factor regions S1 (and
+// S2 for SwiGLU), each [n][f] and 256-byte aligned.
+struct SavedLayout {
+    size_t h = 0, s = 0;
+    int nfac = 1;
+    size_t total() const { return h + nfac * s; }
+};
+
+SavedLayout saved_layout(int64_t n, int64_t f, tsp_act_t act) {
+    SavedLayout l;
+    l.h = align256(static_cast<size_t>(n) * f * 2);
+    l.s = align256(static_cast<size_t>(n) * f * 4);
+    l.nfac = act == TSP_ACT_SWIGLU ? 2 : 1;
+    return l;
+}
+
+// Token rows a launch pair of the training forward covers: the row groups of
+// the pass schedule (at most kRowGroupBudget of H, equal multiples of 256
+// rows), else all rows.
+int64_t train_row_group(int64_t n, int64_t f) {
+    const size_t per_row = static_cast<size_t>(f) * 2;
+    const int64_t cap = static_cast<int64_t>(kRowGroupBudget / per_row) / 256 * 256;
+    if (static_cast<size_t>(n) * per_row <= kRowGroupBudget || cap < 256) return n;
+    const int64_t groups = (n + cap - 1) / cap;
+    return ((n + groups - 1) / groups + 255) / 256 * 256;
+}
+
+template <int ACT>
+tsp_status_t forward_train_bf16(const void* X, const void* Wg, const void* Wu, const void* Wd,
+                                int64_t n, int64_t d, int64_t f, int P, void* Y, void* saved,
+                                cudaStream_t st, int dev, int sms) {
+    const SavedLayout sl = saved_layout(n, f, ACT == 1 ? TSP_ACT_SWIGLU : TSP_ACT_GELU);
+    char* base = static_cast<char*>(saved);
+    auto* H = reinterpret_cast<__nv_bfloat16*>(base);
+    auto* S1 = reinterpret_cast<float*>(base + sl.h);
+    float* S2 = ACT == 1 ? reinterpret_cast<float*>(base + sl.h + sl.s) : nullptr;
+    const int64_t fs = f / P, rg = train_row_group(n, f);
+    const size_t xe = static_cast<size_t>(d) * 2;
+    for (int64_t r0 = 0; r0 < n; r0 += rg) {
+        const int64_t rows = std::min<int64_t>(rg, n - r0);
+        const void* Xg = static_cast<const char*>(X) + r0 * xe;
+        void* Yg = static_cast<char*>(Y) + r0 * xe;
+        const SegGeom g = seg_all_rows(rows, P, fs, 0);
+        const int64_t ho = r0 * f;
+        TSP_TRY(fwd_pass_bf16<ACT>(Xg, Wg, Wu, Wd, rows, d, f, g, f, /*mode direct*/ 3, H + ho,
+                                   nullptr, Yg, st, dev, sms, 0, S1 + ho, S2 ? S2 + ho : nullptr));
+    }
+    return TSP_OK;
+}
+
 // Grid of TM x TM output tiles over rows x cols for each segment.
 template <int TM>
 dim3 f32_grid(int64_t cols, int rows, int segs) {
@@ -894,10 +959,13 @@ struct BwdPlan {
     }
 };
 
-BwdPlan plan_backward_budget(int64_t n, int64_t d, int64_t f, int P, tsp_act_t act, size_t budget) {
+// saved: the backward from the training forward's activations, which needs
+// only the dG (dU) chunk buffers -- no H, no fp32 dH.
+BwdPlan plan_backward_budget(int64_t n, int64_t d, int64_t f, int P, tsp_act_t act, size_t budget,
+                             bool saved) {
     BwdPlan pl;
-    pl.n16 = act == TSP_ACT_SWIGLU ? 3 : 2;
-    pl.n32 = 1;
+    pl.n16 = (act == TSP_ACT_SWIGLU ? 3 : 2) - (saved ? 1 : 0);
+    pl.n32 = saved ? 0 : 1;
     const size_t per_col = static_cast<size_t>(n) * (2 * pl.n16 + 4 * pl.n32);
     const int64_t mc = max_chunk_cols(budget, per_col);
     if (mc == 0) {
@@ -913,41 +981,72 @@ BwdPlan plan_backward_budget(int64_t n, int64_t d, int64_t f, int P, tsp_act_t a
     return pl;
 }
 
-BwdPlan plan_backward(int64_t n, int64_t d, int64_t f, int P, tsp_act_t act) {
-    return plan_backward_budget(n, d, f, P, act, kBwdHiddenBudget);
+BwdPlan plan_backward(int64_t n, int64_t d, int64_t f, int P, tsp_act_t act, bool saved) {
+    return plan_backward_budget(n, d, f, P, act, kBwdHiddenBudget, saved);
 }
 
-BwdPlan plan_backward_for(int64_t n, int64_t d, int64_t f, int P, tsp_act_t act, size_t ws_bytes) {
-    BwdPlan pl = plan_backward(n, d, f, P, act);
+BwdPlan plan_backward_for(int64_t n, int64_t d, int64_t f, int P, tsp_act_t act, size_t ws_bytes,
+                          bool saved) {
+    BwdPlan pl = plan_backward(n, d, f, P, act, saved);
     if (pl.total() <= ws_bytes) return pl;
     const size_t acc = align256(static_cast<size_t>(n) * d * 4);
     if (ws_bytes <= acc + 2048) {
         pl.ok = false;
         return pl;
     }
-    pl = plan_backward_budget(n, d, f, P, act, ws_bytes - acc - 2048);
+    pl = plan_backward_budget(n, d, f, P, act, ws_bytes - acc - 2048, saved);
     if (pl.total() > ws_bytes) pl.ok = false;
     return pl;
 }
+
+// Activations kept by the training forward (see SavedLayout), row pitch ld.
+struct SavedAct {
+    const __nv_bfloat16* H;
+    const float* S1;
+    const float* S2;
+    int64_t ld;
+};
 
 template <int ACT>
 tsp_status_t backward_bf16(const void* X, const void* Wg, const void* Wu, const void* Wd,
                            const void* dY, int64_t n, int64_t d, int64_t f, int P,
                            const BwdPlan& pl, void* dX, float* dWg, float* dWu, float* dWd,
-                           void* ws, cudaStream_t st, int dev, int sms) {
+                           void* ws, cudaStream_t st, int dev, int sms,
+                           const SavedAct* sv = nullptr) {
     char* w = static_cast<char*>(ws);
     const size_t a16 = align256(pl.b16), a32 = align256(pl.b32);
-    auto* Hc = reinterpret_cast<__nv_bfloat16*>(w);
-    auto* dGc = reinterpret_cast<__nv_bfloat16*>(w + a16);
-    auto* dUc = ACT == 1 ? reinterpret_cast<__nv_bfloat16*>(w + 2 * a16) : nullptr;
-    auto* dHc = reinterpret_cast<float*>(w + pl.n16 * a16);
+    int slot = 0;
+    auto* Hc = sv ? nullptr : reinterpret_cast<__nv_bfloat16*>(w + a16 * slot++);
+    auto* dGc = reinterpret_cast<__nv_bfloat16*>(w + a16 * slot++);
+    auto* dUc = ACT == 1 ? reinterpret_cast<__nv_bfloat16*>(w + a16 * slot++) : nullptr;
+    auto* dHc = sv ? nullptr : reinterpret_cast<float*>(w + pl.n16 * a16);
     float* acc = pl.acc_bytes ? reinterpret_cast<float*>(w + pl.n16 * a16 + pl.n32 * a32) : nullptr;
     const int64_t fs = f / P;
     const int np = static_cast<int>(pl.chunks.size());
     for (int i = 0; i < np; ++i) {
         const int64_t cb = pl.chunks[i].col_base, C = pl.chunks[i].width;
+        if (sv) {
+            // K3 from the saved factors: dH = dY . W_down[chunk]^T, applied to
+            // S1 (S2) in the epilogue, giving dG (dU) directly
+            DhFactorParams p;
+            std::memset(&p, 0, sizeof(p));
+            if (!tmap_bf16(&p.tmDY, dY, d, n, d, 64, 128, SW128) ||
+                !tmap_bf16(&p.tmD, Wd, d, f, d, 64, 128, SW128))
+                return TSP_ERR_CUDA;
+            p.n = static_cast<int>(n);
+            p.d = static_cast<int>(d);
+            p.col_base = static_cast<int>(cb);
+            p.width = static_cast<int>(C);
+            p.ld = C;
+            p.S1 = sv->S1 + cb;
+            p.S2 = ACT == 1 ? sv->S2 + cb : nullptr;
+            p.lds = sv->ld;
+            p.dG = dGc;
+            p.dU = dUc;
+            TSP_TRY(launch_pair<DhFactorPair<ACT>>(p, st, dev, sms));
+        }
         // K3a: dH = dY . W_down[chunk]^T, kept in fp32
-        {
+        if (!sv) {
             DhParams p;
             std::memset(&p, 0, sizeof(p));
             if (!tmap_bf16(&p.tmDY, dY, d, n, d, 64, 128, SW128) ||
@@ -962,7 +1061,7 @@ tsp_status_t backward_bf16(const void* X, const void* Wg, const void* Wu, const 
             TSP_TRY(launch_pair<DhPair<ACT>>(p, st, dev, sms));
         }
         // K3b: recompute G (U); emit H and, from dH, dG (dU)
-        {
+        if (!sv) {
             BwdGateUpParams p;
             std::memset(&p, 0, sizeof(p));
             if (!tmap_bf16(&p.tmX, X, d, n, d, 64, 128, SW128) ||
@@ -985,7 +1084,9 @@ tsp_status_t backward_bf16(const void* X, const void* Wg, const void* Wu, const 
             using K = Wgrad<256, false>;
             typename K::Params p;
             std::memset(&p, 0, sizeof(p));
-            if (!tmap_bf16(&p.tmA, Hc, C, n, C, 64, 64, SW128) ||
+            // H: the recomputed chunk, or the chunk's columns of the saved H
+            const __nv_bfloat16* Hs = sv ? sv->H + cb : Hc;
+            if (!tmap_bf16(&p.tmA, Hs, C, n, sv ? sv->ld : C, 64, 64, SW128) ||
                 !tmap_bf16(&p.tmB0, dY, d, n, d, 64, 64, SW128))
                 return TSP_ERR_CUDA;
             p.ntok = static_cast<int>(n);
@@ -1114,7 +1215,7 @@ tsp_status_t tsp_mlp_workspace_size(int64_t n, int64_t d, int64_t f, int P, tsp_
     TSP_TRY(validate_shape(n, d, f, P, act, dt, sched));
     if (backward) {
         if (dt != TSP_DT_BF16 || sched != TSP_SCHED_WEIGHT_SHARDS) return TSP_ERR_INVALID_ARG;
-        *bytes = plan_backward(n, d, f, P, act).total();
+        *bytes = plan_backward(n, d, f, P, act, false).total();
     } else {
         *bytes = plan_forward(n, d, f, P, dt, sched).total();
     }
@@ -1173,7 +1274,7 @@ tsp_status_t tsp_mlp_backward_ex(const void* X, const void* Wg, const void* Wu, 
                                  tsp_act_t act, void* dX, float* dWg, float* dWu, float* dWd,
                                  void* ws, size_t ws_bytes, tsp_stream_t stream) {
     TSP_TRY(validate_backward(X, Wg, Wu, Wd, dY, n, d, f, P, act, dX, dWg, dWu, dWd));
-    const BwdPlan pl = plan_backward_for(n, d, f, P, act, ws ? ws_bytes : 0);
+    const BwdPlan pl = plan_backward_for(n, d, f, P, act, ws ? ws_bytes : 0, false);
     const size_t need = pl.total();
     if (!pl.ok || !ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u))
         return TSP_ERR_WORKSPACE;
@@ -1198,7 +1299,7 @@ tsp_status_t tsp_mlp_backward(const void* X, const void* Wg, const void* Wu, con
                               tsp_act_t act, void* dX, float* dWg, float* dWu, float* dWd,
                               tsp_stream_t stream) {
     TSP_TRY(validate_backward(X, Wg, Wu, Wd, dY, n, d, f, P, act, dX, dWg, dWu, dWd));
-    const size_t need = plan_backward(n, d, f, P, act).total();
+    const size_t need = plan_backward(n, d, f, P, act, false).total();
     int dev = 0;
     DevInfo di;
     TSP_TRY(current_device(&dev, &di));
@@ -1209,6 +1310,84 @@ tsp_status_t tsp_mlp_backward(const void* X, const void* Wg, const void* Wu, con
                                                dWd, ws, need, stream);
     if (cudaFreeAsync(ws, st) != cudaSuccess && s == TSP_OK) return TSP_ERR_CUDA;
     return s;
+}
+
+tsp_status_t tsp_mlp_saved_size(int64_t n, int64_t d, int64_t f, int P, tsp_act_t act,
+                                size_t* bytes) {
+    if (!bytes) return TSP_ERR_INVALID_ARG;
+    TSP_TRY(validate_shape(n, d, f, P, act, TSP_DT_BF16, TSP_SCHED_WEIGHT_SHARDS));
+    *bytes = saved_layout(n, f, act).total();
+    return TSP_OK;
+}
+
+tsp_status_t tsp_mlp_forward_train(const void* X, const void* Wg, const void* Wu, const void* Wd,
+                                   int64_t n, int64_t d, int64_t f, int P, tsp_act_t act, void* Y,
+                                   void* saved, size_t saved_bytes, tsp_stream_t stream) {
+    TSP_TRY(validate_forward(X, Wg, Wu, Wd, n, d, f, P, act, TSP_DT_BF16,
+                             TSP_SCHED_WEIGHT_SHARDS, Y));
+    const size_t need = saved_layout(n, f, act).total();
+    if (!saved || saved_bytes < need || (reinterpret_cast<uintptr_t>(saved) & 255u))
+        return TSP_ERR_INVALID_ARG;
+    const size_t xb = n * d * 2, wb = d * f * 2;
+    if (overlaps(saved, need, X, xb) || overlaps(saved, need, Wg, wb) ||
+        overlaps(saved, need, Wu, wb) || overlaps(saved, need, Wd, wb) ||
+        overlaps(saved, need, Y, xb))
+        return TSP_ERR_INVALID_ARG;
+    int dev = 0;
+    DevInfo di;
+    TSP_TRY(current_device(&dev, &di));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (act == TSP_ACT_SWIGLU)
+        return forward_train_bf16<1>(X, Wg, Wu, Wd, n, d, f, P, Y, saved, st, dev, di.sms);
+    return forward_train_bf16<0>(X, Wg, Wu, Wd, n, d, f, P, Y, saved, st, dev, di.sms);
+}
+
+tsp_status_t tsp_mlp_backward_saved_workspace_size(int64_t n, int64_t d, int64_t f, int P,
+                                                   tsp_act_t act, size_t* bytes) {
+    if (!bytes) return TSP_ERR_INVALID_ARG;
+    TSP_TRY(validate_shape(n, d, f, P, act, TSP_DT_BF16, TSP_SCHED_WEIGHT_SHARDS));
+    *bytes = plan_backward(n, d, f, P, act, true).total();
+    return TSP_OK;
+}
+
+tsp_status_t tsp_mlp_backward_saved(const void* X, const void* Wg, const void* Wu, const void* Wd,
+                                    const void* dY, const void* saved, size_t saved_bytes,
+                                    int64_t n, int64_t d, int64_t f, int P, tsp_act_t act,
+                                    void* dX, float* dWg, float* dWu, float* dWd, void* ws,
+                                    size_t ws_bytes, tsp_stream_t stream) {
+    TSP_TRY(validate_backward(X, Wg, Wu, Wd, dY, n, d, f, P, act, dX, dWg, dWu, dWd));
+    const SavedLayout sl = saved_layout(n, f, act);
+    if (!saved || saved_bytes < sl.total() || (reinterpret_cast<uintptr_t>(saved) & 255u))
+        return TSP_ERR_INVALID_ARG;
+    const BwdPlan pl = plan_backward_for(n, d, f, P, act, ws ? ws_bytes : 0, true);
+    const size_t need = pl.total();
+    if (!pl.ok || !ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u))
+        return TSP_ERR_WORKSPACE;
+    const size_t xb = n * d * 2, wb = d * f * 2, gw = d * f * 4;
+    const void* outs[4] = {dX, dWg, dWu, dWd};
+    const size_t osz[4] = {xb, gw, gw, gw};
+    for (int i = 0; i < 4; ++i)
+        if (overlaps(saved, sl.total(), outs[i], osz[i])) return TSP_ERR_INVALID_ARG;
+    if (overlaps(saved, sl.total(), ws, need)) return TSP_ERR_INVALID_ARG;
+    const void* bufs[9] = {X, Wg, Wu, Wd, dY, dX, dWg, dWu, dWd};
+    const size_t sz[9] = {xb, wb, wb, wb, xb, xb, gw, gw, gw};
+    for (int i = 0; i < 9; ++i)
+        if (overlaps(ws, need, bufs[i], sz[i])) return TSP_ERR_INVALID_ARG;
+    int dev = 0;
+    DevInfo di;
+    TSP_TRY(current_device(&dev, &di));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const char* base = static_cast<const char*>(saved);
+    const SavedAct sv{reinterpret_cast<const __nv_bfloat16*>(base),
+                      reinterpret_cast<const float*>(base + sl.h),
+                      act == TSP_ACT_SWIGLU ? reinterpret_cast<const float*>(base + sl.h + sl.s)
+                                            : nullptr,
+                      f};
+    if (act == TSP_ACT_SWIGLU)
+        return backward_bf16<1>(X, Wg, Wu, Wd, dY, n, d, f, P, pl, dX, dWg, dWu, dWd, ws, st, dev,
+                                di.sms, &sv);
+    return backward_bf16<0>(X, Wg, Wu, Wd, dY, n, d, f, P, pl, dX, dWg, dWu, dWd, ws, st, dev,
+                            di.sms, &sv);
 }
 
 tsp_status_t tsp_trace_enable(int enable) {

@@ -30,7 +30,9 @@ def lib():
 def test_header_declares_the_api():
     syms = set(declared_symbols())
     assert {"tsp_mlp_forward", "tsp_mlp_forward_ex", "tsp_mlp_backward", "tsp_mlp_backward_ex",
-            "tsp_mlp_workspace_size", "tsp_status_string", "tsp_poll_device_error"} <= syms
+            "tsp_mlp_workspace_size", "tsp_status_string", "tsp_poll_device_error",
+            "tsp_mlp_saved_size", "tsp_mlp_forward_train", "tsp_mlp_backward_saved",
+            "tsp_mlp_backward_saved_workspace_size"} <= syms
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -155,6 +157,57 @@ def test_bad_pointers_are_rejected_before_any_device_call(lib):
                               stream=0, check=False) == 1
     assert T.tsp_mlp_backward_ex(X, A, U, B, Y, 64, 64, 128, 1, "swiglu", dX, g1, g1, g3,
                                  0xB00000, 1 << 30, stream=0, check=False) == 1
+
+
+def test_training_pair_sizes(lib):
+    # saved activations: bf16 H, then fp32 S1 (and S2 for SwiGLU), each region
+    # 256-byte aligned
+    n, d, f, P = 4096, 4096, 14336, 8
+    assert T.tsp_mlp_saved_size(n, d, f, P, "swiglu") == n * f * 2 + 2 * n * f * 4
+    assert T.tsp_mlp_saved_size(n, d, f, P, "gelu") == n * f * 2 + n * f * 4
+    assert T.tsp_mlp_saved_size(3, 16, 8 * 3, 3, "swiglu") == \
+        _a256(3 * 24 * 2) + 2 * _a256(3 * 24 * 4)
+    # the backward from saved activations needs only dG (dU) chunk buffers:
+    # one chunk of all hidden units within the 1 GiB budget
+    assert T.tsp_mlp_backward_saved_workspace_size(n, d, f, P, "swiglu") == 2 * n * f * 2
+    assert T.tsp_mlp_backward_saved_workspace_size(n, d, f, P, "gelu") == n * f * 2
+    # 32768 tokens: 2 x 32768 x 14336 x 2 B is above 1 GiB, so chunks of whole
+    # shards (4 of the 8) plus the fp32 dX accumulator
+    n2 = 32768
+    ws = T.tsp_mlp_backward_saved_workspace_size(n2, d, f, P, "swiglu")
+    per_col = n2 * 2 * 2
+    cols = (1 << 30) // per_col // 128 * 128
+    G = max(g for g in (1, 2, 4, 8) if g * (f // P) <= cols)
+    assert ws == 2 * n2 * G * (f // P) * 2 + n2 * d * 4
+
+
+def test_training_pair_rejects_bad_buffers(lib):
+    A, B, X, Y, U = 0x100000, 0x200000, 0x300000, 0x400000, 0x500000
+    n, d, f, P = 64, 64, 128, 1
+    need = T.tsp_mlp_saved_size(n, d, f, P, "swiglu")
+    S = 0x1000000
+    fw = T.tsp_mlp_forward_train
+    assert fw(X, A, U, B, n, d, f, P, "swiglu", Y, None, need, stream=0, check=False) == 1
+    assert fw(X, A, U, B, n, d, f, P, "swiglu", Y, S, need - 1, stream=0, check=False) == 1
+    assert fw(X, A, U, B, n, d, f, P, "swiglu", Y, S + 16, need, stream=0, check=False) == 1
+    assert fw(X, A, U, B, n, d, f, P, "swiglu", Y, X, need, stream=0, check=False) == 1
+    assert fw(X, A, None, B, n, d, f, P, "swiglu", Y, S, need, stream=0, check=False) == 1
+    dX, g1, g2, g3, W = 0x600000, 0x700000, 0x800000, 0xA00000, 0x2000000
+    ws = T.tsp_mlp_backward_saved_workspace_size(n, d, f, P, "swiglu")
+    bw = T.tsp_mlp_backward_saved
+    assert bw(X, A, U, B, Y, None, need, n, d, f, P, "swiglu", dX, g1, g2, g3, W, ws, stream=0,
+              check=False) == 1
+    assert bw(X, A, U, B, Y, S, need - 1, n, d, f, P, "swiglu", dX, g1, g2, g3, W, ws, stream=0,
+              check=False) == 1
+    assert bw(X, A, U, B, Y, S, need, n, d, f, P, "swiglu", dX, g1, g2, g3, None, 0, stream=0,
+              check=False) == 6
+    assert bw(X, A, U, B, Y, S, need, n, d, f, P, "swiglu", dX, g1, g2, g3, W, 16, stream=0,
+              check=False) == 6
+    # an output or the workspace inside the saved buffer
+    assert bw(X, A, U, B, Y, S, need, n, d, f, P, "swiglu", S + 256, g1, g2, g3, W, ws, stream=0,
+              check=False) == 1
+    assert bw(X, A, U, B, Y, S, need, n, d, f, P, "swiglu", dX, g1, g2, g3, S, ws, stream=0,
+              check=False) == 1
 
 
 def test_missing_library_fails_loudly(tmp_path):
