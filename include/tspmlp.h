@@ -230,8 +230,9 @@ TSP_API tsp_status_t tsp_mlp_workspace_size(int64_t n_tokens, int64_t d_model, i
  * dW_gate and dW_up are bit-identical to its results; dW_down uses the
  * forward's H.
  *
- * The saved buffer is opaque to the caller: H, then S1, then S2, each region
- * 256-byte aligned; tsp_mlp_saved_size gives its size.  It must be 256-byte
+ * The saved buffer is opaque to the caller: H (row-major), then S1, then S2
+ * (each over whole 32-row blocks, in the layout the two epilogues access
+ * fastest), every region 256-byte aligned; tsp_mlp_saved_size gives its size.  It must be 256-byte
  * aligned and overlap no other argument; the backward only reads it. */
 TSP_API tsp_status_t tsp_mlp_saved_size(int64_t n_tokens, int64_t d_model, int64_t d_ff, int P,
                                         tsp_act_t act, size_t* bytes);

@@ -12,6 +12,12 @@
 // z phi(z) -- the derivatives of the forward definition, evaluated by the
 // recompute backward's own helpers (bwd_pair.cuh, every rounding explicit),
 // so dG and dU come out bit for bit the same.  dH itself is never stored.
+//
+// The factors are private to this pair, so their layout follows the
+// epilogues' access, where a thread owns a row and a warp 32 consecutive rows:
+// factor (r, c) sits at ((r / 32) * ld + c) * 32 + r % 32, each 32-row block
+// column-interleaved.  A warp then reads or writes one column of its 32 rows
+// as 128 contiguous bytes, instead of 32 rows' 16-byte pieces.
 #pragma once
 
 #include "bwd_pair.cuh"
@@ -22,9 +28,14 @@ namespace tspmlp {
 // Gate/up projection (as FwdHiddenPair) whose epilogue also keeps S1 (S2).
 template <int ACT>
 struct FwdHiddenSaveParams : FwdHidden<ACT>::Params {
-    float* S1;  // [rows][ldh] fp32, indexed as H
-    float* S2;  // [rows][ldh] fp32 (SwiGLU)
+    float* S1;  // fp32, 32-row blocks of ldh columns, column-interleaved
+    float* S2;  // (SwiGLU)
 };
+
+// Offset of factor (r, c) in the 32-row-block layout with ld columns.
+__device__ __forceinline__ long long factor_index(int r, int c, long long ld) {
+    return (static_cast<long long>(r >> 5) * ld + c) * 32 + (r & 31);
+}
 
 template <int ACT>
 struct FwdHiddenSavePair : FwdHiddenPair<ACT> {
@@ -33,11 +44,19 @@ struct FwdHiddenSavePair : FwdHiddenPair<ACT> {
     using Tile = typename Base::Tile;
     static constexpr const char* kName = ACT == 1 ? "fwd_hidden_swiglu_save" : "fwd_hidden_gelu_save";
 
+    // the thread's 32 consecutive factors of one row: a column 32 floats apart
+    __device__ static void store_factors(float* dst, const uint32_t (&v)[32], int valid) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            if (i < valid) dst[32 * i] = __uint_as_float(v[i]);
+    }
+
     __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t rank, uint32_t acc,
                                     int q, int lane) {
         const int rl = (2 * ti.mi + static_cast<int>(rank)) * 128 + q * 32 + lane;
         const bool row_ok = rl < p.g.seg_rows;
-        const long long off = static_cast<long long>(ti.s * p.g.seg_rows + rl) * p.ldh;
+        const int r = ti.s * p.g.seg_rows + rl;
+        const long long off = static_cast<long long>(r) * p.ldh;
         const uint32_t t0 = acc + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll 1
         for (int cc = 0; cc < Base::kOut / 32; ++cc) {
@@ -63,8 +82,8 @@ struct FwdHiddenSavePair : FwdHiddenPair<ACT> {
                 for (int i = 0; i < 16; ++i)
                     pk[i] = pack_bf16x2(__uint_as_float(g[2 * i]), __uint_as_float(g[2 * i + 1]));
                 store_bf16x32(p.H + off + c0, pk, valid);
-                store_f32x32(p.S1 + off + c0, s1, valid);
-                store_f32x32(p.S2 + off + c0, s2, valid);
+                store_factors(p.S1 + factor_index(r, c0, p.ldh), s1, valid);
+                store_factors(p.S2 + factor_index(r, c0, p.ldh), s2, valid);
             } else {
                 tmem_ld_wait();
                 if (!row_ok || valid <= 0) continue;
@@ -79,7 +98,7 @@ struct FwdHiddenSavePair : FwdHiddenPair<ACT> {
                 for (int i = 0; i < 16; ++i)
                     pk[i] = pack_bf16x2(__uint_as_float(g[2 * i]), __uint_as_float(g[2 * i + 1]));
                 store_bf16x32(p.H + off + c0, pk, valid);
-                store_f32x32(p.S1 + off + c0, s1, valid);
+                store_factors(p.S1 + factor_index(r, c0, p.ldh), s1, valid);
             }
         }
     }
@@ -89,9 +108,9 @@ struct FwdHiddenSavePair : FwdHiddenPair<ACT> {
 // dH = dY . W_down[c..]^T (as DhPair), whose epilogue applies the saved
 // factors and writes dG (dU) in bf16 instead of storing dH.
 struct DhFactorParams : DhParams {
-    const float* S1;  // saved factors at the chunk's first column, row pitch lds
+    const float* S1;  // saved factors (32-row-block layout) from the chunk's first column
     const float* S2;  // (SwiGLU)
-    long long lds;
+    long long lds;    // columns of the saved layout (d_ff)
     __nv_bfloat16* dG;  // [n][width] at pitch ld
     __nv_bfloat16* dU;  // [n][width] (SwiGLU)
 };
@@ -103,22 +122,11 @@ struct DhFactorPair : DhPair<ACT> {
     using Tile = typename Base::Tile;
     static constexpr const char* kName = ACT == 1 ? "bwd_dh_factor_swiglu" : "bwd_dh_factor_gelu";
 
-    // 32 fp32 factors from src[0..valid) (zero beyond)
-    __device__ static void load_f32x32(const float* src, int valid, float (&v)[32]) {
-        if (valid >= 32) {
-            const float4* s4 = reinterpret_cast<const float4*>(src);
+    // the thread's 32 consecutive factors of one row (a column 32 floats
+    // apart), zero beyond valid
+    __device__ static void load_factors(const float* src, int valid, float (&v)[32]) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float4 x = s4[i];
-                v[4 * i] = x.x;
-                v[4 * i + 1] = x.y;
-                v[4 * i + 2] = x.z;
-                v[4 * i + 3] = x.w;
-            }
-        } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = i < valid ? src[i] : 0.0f;
-        }
+        for (int i = 0; i < 32; ++i) v[i] = i < valid ? src[32 * i] : 0.0f;
     }
 
     __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t rank, uint32_t acc,
@@ -126,7 +134,6 @@ struct DhFactorPair : DhPair<ACT> {
         const int row = ti.mi * 256 + static_cast<int>(rank) * 128 + q * 32 + lane;
         const bool row_ok = row < p.n;
         const long long off = static_cast<long long>(row) * p.ld;
-        const long long soff = static_cast<long long>(row) * p.lds;
         const uint32_t t0 = acc + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll 1
         for (int cc = 0; cc < 8; ++cc) {
@@ -135,8 +142,9 @@ struct DhFactorPair : DhPair<ACT> {
             const bool live = row_ok && valid > 0;
             float s1[32], s2[32];
             if (live) {
-                load_f32x32(p.S1 + soff + c0, valid, s1);
-                if (ACT == 1) load_f32x32(p.S2 + soff + c0, valid, s2);
+                const long long so = factor_index(row, c0, p.lds);
+                load_factors(p.S1 + so, valid, s1);
+                if (ACT == 1) load_factors(p.S2 + so, valid, s2);
             }
             uint32_t dh[32], pk[16];
             tmem_ld_32x32b_x32(t0 + 32 * cc, dh);

@@ -835,7 +835,8 @@ tsp_status_t forward_bf16(const void* X, const void* Wg, const void* Wu, const v
 // training forward: the weight-shard pass schedule with its activations kept
 
 // Saved activations: H (bf16 [n][f]), then the fp32 factor regions S1 (and
-// S2 for SwiGLU), each [n][f] and 256-byte aligned.
+// S2 for SwiGLU), each of whole 32-row blocks of f columns (the layout of
+// train_pair.cuh), every region 256-byte aligned.
 struct SavedLayout {
     size_t h = 0, s = 0;
     int nfac = 1;
@@ -845,7 +846,7 @@ struct SavedLayout {
 SavedLayout saved_layout(int64_t n, int64_t f, tsp_act_t act) {
     SavedLayout l;
     l.h = align256(static_cast<size_t>(n) * f * 2);
-    l.s = align256(static_cast<size_t>(n) * f * 4);
+    l.s = align256(static_cast<size_t>((n + 31) / 32 * 32) * f * 4);
     l.nfac = act == TSP_ACT_SWIGLU ? 2 : 1;
     return l;
 }
@@ -877,6 +878,8 @@ tsp_status_t forward_train_bf16(const void* X, const void* Wg, const void* Wu, c
         const void* Xg = static_cast<const char*>(X) + r0 * xe;
         void* Yg = static_cast<char*>(Y) + r0 * xe;
         const SegGeom g = seg_all_rows(rows, P, fs, 0);
+        // row groups start on 256-row boundaries, so a group's factors begin
+        // at the same offset r0 x f as its rows of H
         const int64_t ho = r0 * f;
         TSP_TRY(fwd_pass_bf16<ACT>(Xg, Wg, Wu, Wd, rows, d, f, g, f, /*mode direct*/ 3, H + ho,
                                    nullptr, Yg, st, dev, sms, 0, S1 + ho, S2 ? S2 + ho : nullptr));
@@ -1038,8 +1041,8 @@ tsp_status_t backward_bf16(const void* X, const void* Wg, const void* Wu, const 
             p.col_base = static_cast<int>(cb);
             p.width = static_cast<int>(C);
             p.ld = C;
-            p.S1 = sv->S1 + cb;
-            p.S2 = ACT == 1 ? sv->S2 + cb : nullptr;
+            p.S1 = sv->S1 + cb * 32;  // column cb of every 32-row block
+            p.S2 = ACT == 1 ? sv->S2 + cb * 32 : nullptr;
             p.lds = sv->ld;
             p.dG = dGc;
             p.dU = dUc;
