@@ -306,3 +306,39 @@ def mlp_backward(X, W_gate, W_up, W_down, dY, P: int, act: str, workspace=None, 
     tsp_mlp_backward_ex(X, W_gate, W_up, W_down, dY, n, d, f, P, act, dX, dWg, dWu, dWd, ws, need,
                         stream)
     return dX, dWg, dWu, dWd
+
+
+def mlp_forward_train(X, W_gate, W_up, W_down, P: int, act: str, stream=None):
+    """(Y, saved) through tsp_mlp_forward_train (bf16): Y as mlp_forward gives
+    it, and the uint8 buffer of activations that mlp_backward_saved reads."""
+    import torch
+    n, d = X.shape
+    f = W_gate.shape[1]
+    Y = torch.empty((n, d), dtype=torch.bfloat16, device=X.device)
+    need = tsp_mlp_saved_size(n, d, f, P, act)
+    saved = torch.empty(need, dtype=torch.uint8, device=X.device)
+    tsp_mlp_forward_train(X, W_gate, W_up, W_down, n, d, f, P, act, Y, saved, need, stream)
+    return Y, saved
+
+
+def mlp_backward_saved(X, W_gate, W_up, W_down, dY, saved, P: int, act: str, workspace=None,
+                       stream=None):
+    """(dX bf16, dW_gate fp32, dW_up fp32 or None, dW_down fp32) through
+    tsp_mlp_backward_saved, from the buffer mlp_forward_train returned for the
+    same X and weights; a given workspace tensor is passed with its own size."""
+    import torch
+    n, d = X.shape
+    f = W_gate.shape[1]
+    dev = X.device
+    dX = torch.empty((n, d), dtype=torch.bfloat16, device=dev)
+    dWg = torch.empty((d, f), dtype=torch.float32, device=dev)
+    dWu = torch.empty((d, f), dtype=torch.float32, device=dev) if act == "swiglu" else None
+    dWd = torch.empty((f, d), dtype=torch.float32, device=dev)
+    if workspace is None:
+        need = tsp_mlp_backward_saved_workspace_size(n, d, f, P, act)
+        ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    else:
+        ws, need = workspace, _nbytes(workspace)
+    tsp_mlp_backward_saved(X, W_gate, W_up, W_down, dY, saved, _nbytes(saved), n, d, f, P, act, dX,
+                           dWg, dWu, dWd, ws, need, stream)
+    return dX, dWg, dWu, dWd

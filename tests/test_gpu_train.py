@@ -213,3 +213,18 @@ def test_train_pair_writes_nothing_outside_its_buffers(act, n, d, f, P):
     ref = oracle.mlp_backward(inp["X"], inp["A"], inp["Wu"], inp["B"], inp["dY"], act)
     check(np64(dX), ref[0], "dX")
     check(np64(dWd), ref[3], "dW_down")
+
+
+def test_torch_conveniences_match_the_entry_points():
+    n, d, f, P, act = 260, 128, 4 * 128, 4, "swiglu"
+    wl = Workload("train_conv", act, "bf16", n, d, f, P, seed=12, w_std=0.05, backward=True)
+    inp = make_inputs(wl)
+    dev = {k: (v.to("cuda") if v is not None else None) for k, v in inp.items()}
+    Y, saved, g = train_step(dev, n, d, f, P, act)
+    Y2, saved2 = T.mlp_forward_train(dev["X"], dev["A"], dev["Wu"], dev["B"], P, act)
+    g2 = T.mlp_backward_saved(dev["X"], dev["A"], dev["Wu"], dev["B"], dev["dY"], saved2, P, act)
+    torch.cuda.synchronize()
+    assert T.tsp_poll_device_error() == T.TSP_OK
+    assert torch.equal(Y, Y2)
+    for a, b in zip(g, g2):
+        assert torch.equal(a, b)
