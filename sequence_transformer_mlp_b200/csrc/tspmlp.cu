@@ -833,6 +833,14 @@ tsp_status_t forward_bf16(const void* X, const void* Wg, const void* Wu, const v
 
 // ---------------------------------------------------------------------------
 // training forward: the weight-shard pass schedule with its activations kept
+//
+// The block is the gated MLP of "Folding Tensor and Sequence Parallelism for
+// Memory-Efficient Transformer Training & Inference" (Abstract) or the plain
+// one of "Tensor Parallelism: Splitting the Math"; that page notes that the
+// backward pass repeats the forward's split.  The backward needs, per hidden
+// unit, the derivative of the activation at the pre-activation; the forward
+// keeps those factors (train_pair.cuh) so that the backward need not run the
+// gate/up projection again.
 
 // Saved activations: H (bf16 [n][f]), then the fp32 factor regions S1 (and
 // S2 for SwiGLU), each of whole 32-row blocks of f columns (the layout of
