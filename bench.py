@@ -51,6 +51,8 @@ FORWARD_SOURCES = ["ptx.cuh", "pipeline.cuh", "pipeline2.cuh", "recipes.cuh"]
 def kernel_sources(kernel: str) -> list[str]:
     if kernel.endswith("_save") or kernel.startswith("bwd_dh_factor"):
         return FORWARD_SOURCES + ["bwd_pair.cuh", "train_pair.cuh"]
+    if kernel.startswith("dgrad_wgrad"):
+        return FORWARD_SOURCES + ["bwd_pair.cuh", "train_pair.cuh", "grad_pair.cuh"]
     if kernel.startswith("fused_fwd"):
         return FORWARD_SOURCES + ["fused.cuh"]
     if kernel.startswith("fused_passes"):
@@ -521,6 +523,7 @@ def kernel_flops_per_step(kernel: str, wl) -> float:
         "wgrad_gate_up": 2 * 2 * n * d * f,
         "wgrad_gelu_a": 2 * n * d * f,
         "dgrad_accum_swiglu": 2 * 2 * n * d * f,
+        "dgrad_wgrad_swiglu": 2 * 2 * n * d * f + 2 * 2 * n * d * f,
         "dgrad_accum_gelu": 2 * n * d * f,
         "f32_hidden_swiglu": 2 * 2 * n * d * f,
         "f32_hidden_gelu": 2 * n * d * f,

@@ -21,6 +21,7 @@
 #include "../../include/tspmlp.h"
 #include "bwd_pair.cuh"
 #include "train_pair.cuh"
+#include "grad_pair.cuh"
 #include "fused.cuh"
 #include "fused2.cuh"
 #include "pipeline2.cuh"
@@ -1108,6 +1109,39 @@ tsp_status_t backward_bf16(const void* X, const void* Wg, const void* Wu, const 
             p.out_row0 = static_cast<int>(cb);
             p.out_col0 = 0;
             TSP_TRY((launch_pair<WgradPair<256, false>>(p, st, dev, sms)));
+        }
+        if (sv && ACT == 1) {
+            // K4b + K5 in one launch (grad_pair.cuh): the input gradient's long
+            // tiles first, the weight gradients' short ones filling each pair
+            DgradWgradParams p;
+            std::memset(&p, 0, sizeof(p));
+            if (!tmap_bf16(&p.w.tmA, X, d, n, d, 64, 128, SW128) ||
+                !tmap_bf16(&p.w.tmB0, dGc, C, n, C, 64, 128, SW128) ||
+                !tmap_bf16(&p.w.tmB1, dUc, C, n, C, 64, 128, SW128))
+                return TSP_ERR_CUDA;
+            p.w.ntok = static_cast<int>(n);
+            p.w.m_valid = static_cast<int>(d);
+            p.w.n_valid = static_cast<int>(C);
+            p.w.out0 = dWg;
+            p.w.out1 = dWu;
+            p.w.ldo = f;
+            p.w.out_row0 = 0;
+            p.w.out_col0 = static_cast<int>(cb);
+            p.d.g = seg_all_rows(n, P, fs, cb);
+            if (!tmap_bf16(&p.d.tmA0, dGc, C, n, C, 64, 128, SW128) ||
+                !tmap_bf16(&p.d.tmB0, Wg, f, d, f, 64, 128, SW128) ||
+                !tmap_bf16(&p.d.tmA1, dUc, C, n, C, 64, 128, SW128) ||
+                !tmap_bf16(&p.d.tmB1, Wu, f, d, f, 64, 128, SW128))
+                return TSP_ERR_CUDA;
+            p.d.kdim = static_cast<int>(C);
+            p.d.n_out = static_cast<int>(d);
+            p.d.mode = accum_mode(i, np);
+            p.d.acc = acc;
+            p.d.ldacc = d;
+            p.d.out = static_cast<__nv_bfloat16*>(dX);
+            p.d.ldo = d;
+            TSP_TRY(launch_pair<DgradWgradPair>(p, st, dev, sms));
+            continue;
         }
         // K4b: dW_gate (dW_up)[:, cb .. cb+C) = X^T . dG (dU)
         if (ACT == 1) {
