@@ -121,6 +121,12 @@ typedef enum {
 } tsp_sched_t;
 
 /* Forward pass, bf16, weight-shard schedule.
+ * Defined by "Tensor Parallelism: Splitting the Math", walk-through "One
+ * transformer MLP, split across two GPUs", steps 2-6 (A split by columns, the
+ * nonlinearity on each shard's own hidden columns, B split by rows to match,
+ * the shards' partial outputs summed into the exact unsharded Y), and by
+ * "Folding Tensor and Sequence Parallelism ...", Abstract (the gated form;
+ * partial outputs accumulate locally instead of through a collective).
  *   X        [n_tokens][d_model] bf16
  *   W_gate   [d_model][d_ff] bf16 -- A for TSP_ACT_GELU
  *   W_up     [d_model][d_ff] bf16 -- must be NULL for TSP_ACT_GELU
@@ -134,6 +140,10 @@ TSP_API tsp_status_t tsp_mlp_forward(const void* X, const void* W_gate, const vo
                              int64_t d_ff, int P, tsp_act_t act, void* Y, tsp_stream_t stream);
 
 /* Forward pass with every option and a caller workspace.
+ * Defined as tsp_mlp_forward ("Tensor Parallelism: Splitting the Math",
+ * walk-through steps 2-6); the TSP_SCHED_TSP_RING schedules follow "Folding
+ * Tensor and Sequence Parallelism ...", Abstract (weight shards circulate in
+ * a ring while each sequence shard accumulates its partial outputs locally).
  *   dtype      TSP_DT_BF16 (tensor cores) or TSP_DT_F32 (fp32 FMA; any sizes)
  *   sched      a tsp_sched_t (the ring schedules need n % P == 0; the fused
  *              ones bf16; TSP_SCHED_TSP_RING_FUSED also (d_ff / P) % 64 == 0)
@@ -170,7 +180,12 @@ TSP_API tsp_status_t tsp_mlp_forward_ex(const void* X, const void* W_gate, const
  * Arguments, requirements and results are those of tsp_mlp_forward.
  * The first call on a device looks up the array's device address (once per
  * device, with that device current); make that first call before any stream
- * capture.  All calls on a device share the one array and it keeps the last
+ * capture.  If it is also the first call into this library on that device,
+ * CUDA's lazy module loading may load the library's device code there at that
+ * moment -- the static array, the other device globals and the kernels --
+ * which allocates device memory and can synchronise.  Callers with a fixed
+ * memory plan should therefore make one call (any problem size) during their
+ * set-up; later calls allocate nothing.  All calls on a device share the one array and it keeps the last
  * call's contents; calls whose executions overlap on the GPU (different
  * streams, or other threads) race on it and must be serialised by the caller. */
 #define TSP_NOALLOC_SCRATCH_BYTES (32u << 20)
@@ -180,6 +195,14 @@ TSP_API tsp_status_t tsp_mlp_forward_noalloc(const void* X, const void* W_gate, 
                                              void* Y, tsp_stream_t stream);
 
 /* Backward pass, bf16, weight-shard schedule, for upstream gradient dY.
+ * "Tensor Parallelism: Splitting the Math", its paragraph counting the
+ * communication (the forward's pattern happens again in the backward pass):
+ * the gradients are the exact derivatives of the forward of tsp_mlp_forward,
+ * computed shard by shard with the input gradient's partials summed locally
+ * like Y's.  With G = X.W_gate, U = X.W_up, dH = dY.W_down^T:
+ *   SwiGLU: dU = dH SiLU(G), dG = dH U SiLU'(G);  GeLU: dG = dH GeLU'(G);
+ *   dX = dG.W_gate^T (+ dU.W_up^T), dW_gate = X^T.dG, dW_up = X^T.dU,
+ *   dW_down = H^T.dY.
  *   dY        [n_tokens][d_model] bf16
  *   dX        [n_tokens][d_model] bf16, written
  *   dW_gate   [d_model][d_ff] fp32, written (dA for TSP_ACT_GELU)
@@ -194,7 +217,10 @@ TSP_API tsp_status_t tsp_mlp_backward(const void* X, const void* W_gate, const v
                               float* dW_gate, float* dW_up, float* dW_down,
                               tsp_stream_t stream);
 
-/* Backward with a caller workspace (bf16 only; weight-shard schedule).  As for
+/* Backward with a caller workspace (bf16 only; weight-shard schedule).
+ * Defined as tsp_mlp_backward ("Tensor Parallelism: Splitting the Math",
+ * paragraph counting the communication: the same pattern in the backward
+ * pass).  As for
  * tsp_mlp_forward_ex, a workspace smaller than the preferred size is accepted
  * down to one 128-column chunk of the hidden buffers plus the fp32 dX
  * accumulator. */

@@ -47,7 +47,10 @@ struct DgradWgradPair {
     __host__ __device__ static int w_mtiles(const Params& p) { return (p.w.m_valid + 255) / 256; }
     __host__ __device__ static int w_ntiles(const Params& p) { return (p.w.n_valid + kWCols - 1) / kWCols; }
     __host__ __device__ static int n_wgrad(const Params& p) { return w_mtiles(p) * w_ntiles(p); }
-    __host__ __device__ static int kb_dgrad(const Params& p) { return 2 * ((p.d.kdim + kBK - 1) / kBK); }
+    // an input-gradient tile's k-blocks, counted exactly as D::num_kb counts
+    // them (two K segments of ceil(kdim / D::kBK) blocks), for any chunk width
+    static_assert(D::kBK == kBK, "both kinds of tile use the same k-block depth");
+    __host__ __device__ static int kb_dgrad(const Params& p) { return 2 * ((p.d.kdim + D::kBK - 1) / D::kBK); }
     __host__ __device__ static int kb_wgrad(const Params& p) { return (p.w.ntok + kBK - 1) / kBK; }
 
     // Schedule over np pairs.  Pair q first runs input-gradient tiles q,

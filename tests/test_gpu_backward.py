@@ -18,7 +18,7 @@ import torch
 
 import oracle
 import sequence_transformer_mlp_b200 as T
-from workloads import FWD_BWD, Workload, make_inputs, sample_rows
+from workloads import FWD_BWD, Workload, cover_cols, cover_rows, make_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -132,13 +132,18 @@ def test_fwd_bwd_llama8b_shape_sampled():
     dX, dWg, dWu, dWd = T.mlp_backward(dev["X"], dev["A"], dev["Wu"], dev["B"], dev["dY"], wl.P,
                                        wl.act)
     assert T.tsp_poll_device_error() == T.TSP_OK
-    rows = sample_rows(wl.n, 12, wl.seed)
+    # one seeded row in each of the 16 blocks of 256 token rows (every pair row
+    # tile of the forward and of the input gradient), plus rows 0 and 4095
+    rows = cover_rows(wl.n, 256, wl.seed)
     refY = oracle.mlp_sharded(inp["X"][rows], inp["A"], inp["Wu"], inp["B"], wl.act, wl.P)
     check(np64(Y[rows]), refY, "Y rows")
     ref_dx = oracle.mlp_backward(inp["X"][rows], inp["A"], inp["Wu"], inp["B"], inp["dY"][rows],
                                  wl.act, outputs=("dX",))[0]
     check(np64(dX[rows]), ref_dx, "dX rows")
-    cols = sample_rows(wl.f, 14, wl.seed + 1)  # hidden columns, incl. first and last
+    # hidden columns: the first and last of each of the 8 weight shards, plus one
+    # seeded column in each of the 112 blocks of 128 (every 128-column tile of
+    # dW_gate | dW_up, every 256-row tile of dW_down)
+    cols = cover_cols(wl.f, wl.P, 128, wl.seed + 1)
     sub = oracle.mlp_backward(inp["X"], inp["A"][:, cols], inp["Wu"][:, cols], inp["B"][cols, :],
                               inp["dY"], wl.act, outputs=("dA", "dWu", "dB"))
     check(np64(dWg[:, cols]), sub[1], "dW_gate cols")

@@ -16,7 +16,8 @@ import torch
 
 import oracle
 import sequence_transformer_mlp_b200 as T
-from workloads import GELU_F32, LLAMA8B, LLAMA70B, TSP_RING, Workload, make_inputs, sample_rows
+from workloads import (GELU_F32, LLAMA8B, LLAMA70B, TSP_RING, Workload, cover_rows, make_inputs,
+                       sample_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -318,7 +319,10 @@ def test_llama8b_shape_sampled_rows(llama8b, P, sched):
     inp, dev = llama8b
     Y = T.mlp_forward(dev["X"], dev["A"], dev["Wu"], dev["B"], P, "swiglu", sched=sched)
     assert T.tsp_poll_device_error() == T.TSP_OK
-    rows = sample_rows(LLAMA8B.n, 24, LLAMA8B.seed)
+    # one seeded row in each of the 16 blocks of 256 token rows (every pair row
+    # tile of the one row group; every second 128-row tile of the one-CTA fused
+    # schedule), plus rows 0 and 4095
+    rows = cover_rows(LLAMA8B.n, 256, LLAMA8B.seed)
     _sampled_check(LLAMA8B, inp, Y, rows, sched=sched, P=P)
 
 
@@ -328,10 +332,13 @@ def test_tsp_ring_long_context_sampled_rows(sched):
     Y = T.mlp_forward(dev["X"], dev["A"], dev["Wu"], dev["B"], TSP_RING.P, "swiglu",
                       sched=sched)
     assert T.tsp_poll_device_error() == T.TSP_OK
-    # rows from every sequence shard, including each shard's first and last row
+    # one seeded row in each of the 128 blocks of 256 token rows (every pair row
+    # tile of every sequence shard, so every ring group of sequence shards),
+    # plus the first and last row of each of the 8 sequence shards
     ns = TSP_RING.n // TSP_RING.P
-    rows = sorted(set(sample_rows(TSP_RING.n, 16, TSP_RING.seed) +
-                      [s * ns for s in range(TSP_RING.P)] + [s * ns + ns - 1 for s in range(TSP_RING.P)]))
+    rows = cover_rows(TSP_RING.n, 256, TSP_RING.seed,
+                      groups=[(s * ns, (s + 1) * ns) for s in range(TSP_RING.P)])
+    assert len(rows) >= 128
     _sampled_check(TSP_RING, inp, Y, rows, sched=sched)
 
 
@@ -339,5 +346,11 @@ def test_llama70b_shape_sampled_rows():
     inp, dev = _full_inputs(LLAMA70B)
     Y = T.mlp_forward(dev["X"], dev["A"], dev["Wu"], dev["B"], LLAMA70B.P, "swiglu")
     assert T.tsp_poll_device_error() == T.TSP_OK
-    rows = sample_rows(LLAMA70B.n, 8, LLAMA70B.seed)
+    # the 70B shape runs as 4 row groups of 2048 tokens (H of a group is 117 MB):
+    # one seeded row in each of the 32 blocks of 256 rows (every pair row tile
+    # of every group), plus each group's first and last row (0, 2047, 2048,
+    # 4095, 4096, 6143, 6144, 8191)
+    groups = [(g * 2048, (g + 1) * 2048) for g in range(4)]
+    rows = cover_rows(LLAMA70B.n, 256, LLAMA70B.seed, groups=groups)
+    assert {4096, 6143} <= set(rows) and len(rows) >= 32
     _sampled_check(LLAMA70B, inp, Y, rows)

@@ -16,7 +16,7 @@ import torch
 
 import oracle
 import sequence_transformer_mlp_b200 as T
-from workloads import FWD_BWD, Workload, make_inputs, sample_rows
+from workloads import FWD_BWD, Workload, cover_cols, cover_rows, make_inputs, sample_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -150,11 +150,24 @@ def test_train_pair_llama8b_shape():
     torch.cuda.synchronize()
     assert torch.equal(dX, r[0]) and torch.equal(dWg, r[1]) and torch.equal(dWu, r[2])
     del r
-    cols = sample_rows(f, 14, wl.seed + 1)  # hidden columns, incl. first and last
+    # dX, dW_gate, dW_up are bit-identical to the recompute backward (checked
+    # above), whose full-shape samples are compared with the oracle in
+    # test_gpu_backward.py; here they are compared with the oracle as well.
+    # Hidden columns: the first and last of each of the 8 weight shards, plus
+    # one seeded column in each of the 112 blocks of 128 (every 128-column tile
+    # of dW_gate | dW_up, every 256-row tile of dW_down)
+    cols = cover_cols(f, P, 128, wl.seed + 1)
     sub = oracle.mlp_backward(inp["X"], inp["A"][:, cols], inp["Wu"][:, cols], inp["B"][cols, :],
-                              inp["dY"], wl.act, outputs=("dB",))
+                              inp["dY"], wl.act, outputs=("dA", "dWu", "dB"))
+    check(np64(dWg[:, cols]), sub[1], "dW_gate cols")
+    check(np64(dWu[:, cols]), sub[2], "dW_up cols")
     check(np64(dWd[cols, :]), sub[3], "dW_down rows")
-    rows = sample_rows(n, 8, wl.seed)
+    # one seeded row in each of the 16 blocks of 256 token rows (every pair row
+    # tile of the training forward and of the input gradient), plus rows 0, 4095
+    rows = cover_rows(n, 256, wl.seed)
+    ref_dx = oracle.mlp_backward(inp["X"][rows], inp["A"], inp["Wu"], inp["B"], inp["dY"][rows],
+                                 wl.act, outputs=("dX",))[0]
+    check(np64(dX[rows]), ref_dx, "dX rows")
     check(np64(saved_h(saved, n, f)[rows]),
           oracle.mlp_hidden(inp["X"][rows], inp["A"], inp["Wu"], wl.act), "saved H rows")
 

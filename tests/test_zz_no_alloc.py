@@ -7,7 +7,9 @@ allocates nothing.
 The test calls it through the C ABI twice in a row (the second call runs on
 whatever the first left in the shared static array) and checks each result
 against the allocating entry point tsp_mlp_forward, within the bf16 tolerance
-the other tests use.  It sits in a file of its own, collected last, so that a
+the other tests use; the small case is also compared with the fp64 oracle
+directly, with the same bar (max|Y - Yref| <= 1e-2 max|Yref|, relative
+Frobenius error <= 5e-3).  It sits in a file of its own, collected last, so that a
 run stopping at the first failure has run every other test first; it holds no
 state between tests and passes alone in a fresh process too.
 """
@@ -15,6 +17,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import sequence_transformer_mlp_b200 as T
 from workloads import Workload, make_inputs
 
@@ -23,7 +26,7 @@ pytestmark = pytest.mark.gpu
 
 def _close(got, ref, what):
     g = got.float().cpu().double().numpy()
-    r = ref.float().cpu().double().numpy()
+    r = ref if isinstance(ref, np.ndarray) else ref.float().cpu().double().numpy()
     assert np.isfinite(g).all(), what
     mx = np.abs(r).max()
     assert np.abs(g - r).max() <= 1e-2 * mx, what
@@ -43,12 +46,18 @@ def test_noalloc_forward_matches_allocating_forward_twice(act, n, d, f, P):
     X, A, Wu, B = (None if inp[k] is None else inp[k].cuda() for k in ("X", "A", "Wu", "B"))
     ref = torch.empty(n, d, dtype=torch.bfloat16, device="cuda")
     T.tsp_mlp_forward(X, A, Wu, B, n, d, f, P, act, ref)
+    # the fp64 oracle on the small case (the large one is covered through the
+    # allocating forward, which the forward tests compare with the oracle)
+    exact = (oracle.mlp_forward(inp["X"], inp["A"], inp["Wu"], inp["B"], act)
+             if n * d * f <= 1 << 28 else None)
     for call in range(2):
         Y = torch.full((n, d), float("nan"), dtype=torch.bfloat16, device="cuda")
         T.tsp_mlp_forward_noalloc(X, A, Wu, B, n, d, f, P, act, Y)
         torch.cuda.synchronize()
         assert T.tsp_poll_device_error() == T.TSP_OK
         _close(Y, ref, f"call {call}")
+        if exact is not None:
+            _close(Y, exact, f"call {call} vs oracle")
 
 
 def test_noalloc_rejects_problems_beyond_its_static_scratch():

@@ -115,3 +115,35 @@ def sample_rows(n: int, count: int, seed: int) -> list[int]:
     rows = set(torch.randperm(n, generator=g)[:k].tolist())
     rows.update({0, n - 1})
     return sorted(rows)
+
+
+def cover_rows(n: int, block: int, seed: int, groups=()) -> list[int]:
+    """Seeded token rows that touch every launch and tile of a full-size run.
+
+    One seeded row inside every ``block``-row block of [0, n) (a 256-row pair
+    tile, say), plus the first and last row of [0, n) and of every
+    ``(begin, end)`` half-open range in ``groups`` (row groups, sequence
+    shards).  Sorted, without repeats.
+    """
+    g = torch.Generator("cpu").manual_seed(seed + 104729)
+    rows = {0, n - 1}
+    for b0 in range(0, n, block):
+        size = min(block, n - b0)
+        rows.add(b0 + int(torch.randint(size, (1,), generator=g)))
+    for b, e in groups:
+        rows.update({b, e - 1})
+    return sorted(r for r in rows if 0 <= r < n)
+
+
+def cover_cols(f: int, P: int, block: int, seed: int) -> list[int]:
+    """Seeded hidden columns that touch every weight shard and column tile.
+
+    Every shard's first and last column, plus one seeded column inside every
+    ``block``-column block of [0, f).  Sorted, without repeats.
+    """
+    fs = f // P
+    cols = set()
+    for w in range(P):
+        cols.update({w * fs, w * fs + fs - 1})
+    cols.update(cover_rows(f, block, seed))
+    return sorted(cols)
