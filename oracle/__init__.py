@@ -20,6 +20,10 @@ pages each function follows is stated in the C file's header:
   ("Folding Tensor and Sequence Parallelism ...", Abstract).
 * ``mlp_backward``     -- closed-form gradients of the forward definition.
 
+Multi-head self-attention under the TSP schedule (the second runtime schedule
+of "Folding Tensor and Sequence Parallelism ...", Abstract) lives in
+``oracle.attention`` (numpy fp64; its header cites the passages).
+
 Activations: ``"gelu"`` is the exact erf GeLU; ``"swiglu"`` is
 ``SiLU(X.Wg) * (X.Wu)``.  Matrices are row-major ``X[n,d]``, ``A=Wg[d,f]``,
 ``Wu[d,f]``, ``B=Wd[f,d]``.

@@ -147,3 +147,64 @@ def cover_cols(f: int, P: int, block: int, seed: int) -> list[int]:
         cols.update({w * fs, w * fs + fs - 1})
     cols.update(cover_rows(f, block, seed))
     return sorted(cols)
+
+
+# ---------------------------------------------------------------------------
+# TSP attention
+
+
+@dataclasses.dataclass(frozen=True)
+class AttnWorkload:
+    """Multi-head self-attention block under the TSP schedule: n tokens in P
+    sequence shards, n_heads heads of d / n_heads in P parameter shards."""
+    name: str
+    n: int              # tokens
+    d: int              # d_model
+    heads: int
+    P: int              # sequence shards = parameter shards
+    causal: bool
+    seed: int
+    w_std: float
+
+    @property
+    def dh(self) -> int:
+        return self.d // self.heads
+
+    def flops(self) -> dict:
+        """Algorithmic FLOPs: the four projections (2 n d^2 each) and the core
+        (2 d per query-key pair for the scores and 2 d for the weighted values;
+        with the causal mask only the n (n + 1) / 2 visible pairs count)."""
+        pairs = self.n * (self.n + 1) // 2 if self.causal else self.n * self.n
+        return {"projections": 4 * 2 * self.n * self.d * self.d, "core": 4 * pairs * self.d}
+
+
+# Input recipe: one torch.Generator('cpu') seeded with the workload's seed,
+# torch.randn in the order X[n, d] ~ N(0, 1), W_q, W_k, W_v, W_o [d, d] ~
+# N(0, w_std^2), cast (round to nearest even) to bf16.  The long-context shape
+# is the TSP ring workload's (32768 tokens in 8 sequence shards of 4096,
+# d_model 4096) with Llama-3-8B's 32 heads of 128.
+ATTN_WORKLOADS = {
+    "tsp_attn_causal_bf16_n32768_d4096_h32": AttnWorkload(
+        "tsp_attn_causal_bf16_n32768_d4096_h32", 32768, 4096, 32, 8, True, seed=5, w_std=0.02),
+    "tsp_attn_bf16_n32768_d4096_h32": AttnWorkload(
+        "tsp_attn_bf16_n32768_d4096_h32", 32768, 4096, 32, 8, False, seed=6, w_std=0.02),
+}
+TSP_ATTN = ATTN_WORKLOADS["tsp_attn_causal_bf16_n32768_d4096_h32"]
+
+
+def make_attn_inputs(wl: AttnWorkload, seed: int | None = None) -> dict:
+    """Seeded bf16 CPU tensors X, Wq, Wk, Wv, Wo of the workload's shapes."""
+    g = torch.Generator("cpu").manual_seed(wl.seed if seed is None else seed)
+    X = torch.randn(wl.n, wl.d, generator=g)
+    W = [torch.randn(wl.d, wl.d, generator=g).mul_(wl.w_std) for _ in range(4)]
+    out = {"X": X}
+    out.update(zip(("Wq", "Wk", "Wv", "Wo"), W))
+    return {k: v.to(torch.bfloat16).contiguous() for k, v in out.items()}
+
+
+def make_qkv(n: int, d: int, seed: int, std: float = 1.0) -> dict:
+    """Seeded bf16 Q, K, V [n, d] ~ N(0, std^2) for tests of the attention core
+    alone (drawn in the order Q, K, V)."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    return {k: torch.randn(n, d, generator=g).mul_(std).to(torch.bfloat16).contiguous()
+            for k in ("Q", "K", "V")}
