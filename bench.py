@@ -40,7 +40,8 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from workloads import WORKLOADS, LLAMA8B, make_inputs  # noqa: E402
+from workloads import (ATTN_WORKLOADS, LLAMA8B, WORKLOADS, make_attn_inputs,  # noqa: E402
+                       make_inputs)
 
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
 # the csrc headers each kernel is built from (a change to any of them voids its
@@ -61,6 +62,8 @@ def kernel_sources(kernel: str) -> list[str]:
         return FORWARD_SOURCES + ["bwd_pair.cuh"]
     if kernel.startswith("f32_"):
         return ["simt_f32.cuh"]
+    if kernel.startswith("attn_core"):
+        return ["ptx.cuh", "pipeline.cuh", "attn.cuh"]
     return FORWARD_SOURCES
 
 
@@ -413,13 +416,167 @@ def end_to_end(args, inp, dev, step, Y, stream, barrier):
     return e2.elapsed_time(e3) / args.steps, Xh, Yh[0]
 
 
+def setup_mlp(args, wl, T, stream):
+    """The MLP step (forward, or forward+backward) through the C ABI."""
+    inp = make_inputs(wl)
+    dev = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
+    n, d, f, P = wl.n, wl.d, wl.f, wl.P
+    sched = args.sched or wl.sched
+    dt = "f32" if wl.dtype == "f32" else "bf16"
+    tdt = torch.float32 if dt == "f32" else torch.bfloat16
+    Y = torch.empty(n, d, dtype=tdt, device="cuda")
+    saved_act = wl.backward and not args.bwd_recompute
+    if not wl.backward:
+        need = T.tsp_mlp_workspace_size(n, d, f, P, wl.act, dt, sched)
+    elif saved_act:
+        need = T.tsp_mlp_backward_saved_workspace_size(n, d, f, P, wl.act)
+    else:
+        need = T.tsp_mlp_workspace_size(n, d, f, P, wl.act, dt, sched, backward=True)
+    ws = torch.empty(max(need, 1), dtype=torch.uint8, device="cuda")
+    st = {}
+    if wl.backward:
+        st["dX"] = torch.empty(n, d, dtype=torch.bfloat16, device="cuda")
+        st["dWg"] = torch.empty(d, f, dtype=torch.float32, device="cuda")
+        st["dWu"] = (torch.empty(d, f, dtype=torch.float32, device="cuda")
+                     if wl.act == "swiglu" else None)
+        st["dWd"] = torch.empty(f, d, dtype=torch.float32, device="cuda")
+        if saved_act:
+            # the training forward keeps H and the activation's factors for the backward
+            st["n_saved"] = T.tsp_mlp_saved_size(n, d, f, P, wl.act)
+            st["saved"] = torch.empty(st["n_saved"], dtype=torch.uint8, device="cuda")
+        else:
+            st["ws_f"] = torch.empty(
+                max(T.tsp_mlp_workspace_size(n, d, f, P, wl.act, "bf16", sched), 1),
+                dtype=torch.uint8, device="cuda")
+
+    def step(x=dev["X"], y=Y):
+        if saved_act:
+            T.tsp_mlp_forward_train(x, dev["A"], dev["Wu"], dev["B"], n, d, f, P, wl.act, y,
+                                    st["saved"], st["n_saved"], stream)
+            T.tsp_mlp_backward_saved(x, dev["A"], dev["Wu"], dev["B"], dev["dY"], st["saved"],
+                                     st["n_saved"], n, d, f, P, wl.act, st["dX"], st["dWg"],
+                                     st["dWu"], st["dWd"], ws, need, stream)
+            return
+        wsf = st["ws_f"] if wl.backward else ws
+        T.tsp_mlp_forward_ex(x, dev["A"], dev["Wu"], dev["B"], n, d, f, P, wl.act, dt, sched,
+                             y, wsf, wsf.numel() if wl.backward else need, stream)
+        if wl.backward:
+            T.tsp_mlp_backward_ex(x, dev["A"], dev["Wu"], dev["B"], dev["dY"], n, d, f, P,
+                                  wl.act, st["dX"], st["dWg"], st["dWu"], st["dWd"], ws, need,
+                                  stream)
+
+    config = {"workload": wl.name, "n_tokens": n, "d_model": d, "d_ff": f, "P": P,
+              "act": wl.act, "schedule": sched,
+              **({"backward": "saved activations" if saved_act else "recompute"}
+                 if wl.backward else {}),
+              "l2": "inputs larger than L2 (weights 3 x d x f bf16), no flush"
+              if dt == "bf16" else "inputs fit in L2 (launch-latency bound), no flush"}
+    return {"step": step, "inp": inp, "dev": dev, "Y": Y, "flops": workload_flops(wl),
+            "dt": dt, "metric": metric_name(wl), "config": config,
+            "kernel_flops": lambda k: kernel_flops_per_step(k, wl),
+            "cpu_baseline": lambda: cpu_baseline(wl), "tokens": n}
+
+
+def setup_attn(args, wl, T, stream):
+    """The TSP attention block's forward through the C ABI."""
+    inp = make_attn_inputs(wl)
+    dev = {k: v.cuda() for k, v in inp.items()}
+    n, d = wl.n, wl.d
+    Y = torch.empty(n, d, dtype=torch.bfloat16, device="cuda")
+    need = T.tsp_attn_workspace_size(n, d, wl.heads, wl.P)
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+
+    def step(x=dev["X"], y=Y):
+        T.tsp_attn_forward(x, dev["Wq"], dev["Wk"], dev["Wv"], dev["Wo"], n, d, wl.heads, wl.P,
+                           wl.causal, y, ws, need, stream)
+
+    fl = wl.flops()
+    per_kernel = {"attn_core": fl["core"], "attn_core_causal": fl["core"],
+                  "attn_proj": fl["projections"] * 3 / 4, "attn_out_proj": fl["projections"] / 4}
+    config = {"workload": wl.name, "n_tokens": n, "d_model": d, "n_heads": wl.heads,
+              "head_dim": wl.dh, "P": wl.P, "causal": wl.causal, "schedule": "tsp_attention",
+              "l2": "inputs larger than L2 (X 268 MB, K/V of one head 16 MB), no flush"}
+    return {"step": step, "inp": inp, "dev": dev, "Y": Y,
+            "flops": fl["core"] + fl["projections"], "dt": "bf16",
+            "metric": "TSP attention forward TFLOP/s", "config": config,
+            "kernel_flops": lambda k: per_kernel[k],
+            "cpu_baseline": lambda: attn_cpu_baseline(wl), "tokens": n}
+
+
+def attn_oracle_sample(wl, inp, rows: int) -> dict:
+    """The fp64 attention oracle, as it stands, on the first `rows` query rows
+    of the block (every key and value of the sequence is projected for them),
+    and the full step's CPU time extrapolated linearly in the number of query
+    rows from two sample sizes."""
+    from oracle import attention as OA
+    args = [inp[k] for k in ("X", "Wq", "Wk", "Wv", "Wo")]
+    times = {}
+    for r in (max(1, rows // 4), rows):
+        t0 = time.perf_counter()
+        OA.attention_forward(*args, wl.heads, wl.causal, rows=list(range(r)))
+        times[r] = time.perf_counter() - t0
+    (r1, t1), (r2, t2) = sorted(times.items())
+    per_row = max((t2 - t1) / max(r2 - r1, 1), 0.0)
+    fixed = max(t1 - per_row * r1, 0.0)
+    return {"rows_s": t2, "fixed_s": fixed, "per_row_s": per_row,
+            "extrapolated_full_step_s": fixed + per_row * wl.n}
+
+
+def attn_cpu_baseline(wl, rows=64):
+    import oracle
+    inp = make_attn_inputs(wl)
+    parts = attn_oracle_sample(wl, inp, rows)
+    full = parts["extrapolated_full_step_s"]
+    fl = wl.flops()
+    return {"value": (fl["core"] + fl["projections"]) / full / 1e12, "unit": "TFLOP/s",
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"first {rows // 4} and {rows} query rows of {wl.name} (fp64 oracle: the "
+                      f"keys and values of all {wl.n} tokens, then attention of those rows); "
+                      f"full step extrapolated linearly in rows: {full:.1f} s",
+            "extrapolated_full_step_s": full}
+
+
+def attn_reference_arm(args, wl, rank):
+    if rank != 0:
+        return
+    import oracle
+    inp = make_attn_inputs(wl)
+    rows = args.ref_rows or 64
+    for _ in range(args.warmup):
+        attn_oracle_sample(wl, inp, rows)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        parts = attn_oracle_sample(wl, inp, rows)
+    dt = (time.perf_counter() - t0) / args.steps
+    fl = wl.flops()
+    full = parts["extrapolated_full_step_s"]
+    tflops = (fl["core"] + fl["projections"]) / full / 1e12
+    line = {
+        "impl": "reference", "metric": "TSP attention forward TFLOP/s", "value": tflops,
+        "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded torch.randn)",
+        "tokens_per_s": wl.n / full,
+        "config": {"workload": wl.name, "n_tokens": wl.n, "d_model": wl.d, "n_heads": wl.heads,
+                   "P": wl.P, "causal": wl.causal, "sample_rows": rows},
+        "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                         "kind": "oracle",
+                         "sample": f"first {rows // 4} and {rows} query rows per step",
+                         "extrapolated_full_step_s": full},
+        "e2e": {"value": tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default=LLAMA8B.name, choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default=LLAMA8B.name,
+                    choices=sorted(WORKLOADS) + sorted(ATTN_WORKLOADS))
     ap.add_argument("--sched", default=None,
                     choices=["weight_shards", "tsp_ring", "shard_passes", "fused", "tsp_ring_fused",
                              "shard_passes_fused"],
@@ -432,12 +589,13 @@ def main():
                          "that keeps its activations")
     ap.add_argument("--ref-rows", type=int, default=None,
                     help="--impl reference: token rows (and, fwd+bwd, hidden columns) of the "
-                         "oracle's sample per step (default 256, 64 for fwd+bwd)")
+                         "oracle's sample per step (default 256, 64 for fwd+bwd and attention)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the host-buffer loop (used for short profiler runs)")
     args = ap.parse_args()
-    wl = WORKLOADS[args.workload]
+    attn = args.workload in ATTN_WORKLOADS
+    wl = ATTN_WORKLOADS[args.workload] if attn else WORKLOADS[args.workload]
     # traffic figures in the committed ncu summaries are for the workload's own P
     traffic_key = wl.name
     if args.P is not None and args.P != wl.P:
@@ -449,7 +607,7 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
 
     if args.impl == "reference":
-        reference_arm(args, wl, rank)
+        (attn_reference_arm if attn else reference_arm)(args, wl, rank)
         return
 
     import sequence_transformer_mlp_b200 as T
@@ -465,50 +623,9 @@ def main():
         if dist is not None:
             dist.barrier()
 
-    inp = make_inputs(wl)
-    dev = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
-    n, d, f, P = wl.n, wl.d, wl.f, wl.P
-    sched = args.sched or wl.sched
     stream = torch.cuda.current_stream()
-    dt = "f32" if wl.dtype == "f32" else "bf16"
-    tdt = torch.float32 if dt == "f32" else torch.bfloat16
-    Y = torch.empty(n, d, dtype=tdt, device="cuda")
-    saved_act = wl.backward and not args.bwd_recompute
-    if not wl.backward:
-        need = T.tsp_mlp_workspace_size(n, d, f, P, wl.act, dt, sched)
-    elif saved_act:
-        need = T.tsp_mlp_backward_saved_workspace_size(n, d, f, P, wl.act)
-    else:
-        need = T.tsp_mlp_workspace_size(n, d, f, P, wl.act, dt, sched, backward=True)
-    ws = torch.empty(max(need, 1), dtype=torch.uint8, device="cuda")
-    if wl.backward:
-        dX = torch.empty(n, d, dtype=torch.bfloat16, device="cuda")
-        dWg = torch.empty(d, f, dtype=torch.float32, device="cuda")
-        dWu = torch.empty(d, f, dtype=torch.float32, device="cuda") if wl.act == "swiglu" else None
-        dWd = torch.empty(f, d, dtype=torch.float32, device="cuda")
-        if saved_act:
-            # the training forward keeps H and the activation's factors for the backward
-            n_saved = T.tsp_mlp_saved_size(n, d, f, P, wl.act)
-            saved = torch.empty(n_saved, dtype=torch.uint8, device="cuda")
-        else:
-            ws_f = torch.empty(max(T.tsp_mlp_workspace_size(n, d, f, P, wl.act, "bf16", sched), 1),
-                               dtype=torch.uint8, device="cuda")
-
-    def step(x=dev["X"], y=Y):
-        if saved_act:
-            T.tsp_mlp_forward_train(x, dev["A"], dev["Wu"], dev["B"], n, d, f, P, wl.act, y, saved,
-                                    n_saved, stream)
-            T.tsp_mlp_backward_saved(x, dev["A"], dev["Wu"], dev["B"], dev["dY"], saved, n_saved,
-                                     n, d, f, P, wl.act, dX, dWg, dWu, dWd, ws, need, stream)
-            return
-        T.tsp_mlp_forward_ex(x, dev["A"], dev["Wu"], dev["B"], n, d, f, P, wl.act, dt, sched,
-                             y, ws_f if wl.backward else ws,
-                             ws_f.numel() if wl.backward else need, stream)
-        if wl.backward:
-            T.tsp_mlp_backward_ex(x, dev["A"], dev["Wu"], dev["B"], dev["dY"], n, d, f, P, wl.act,
-                                  dX, dWg, dWu, dWd, ws, need, stream)
-
-    flops = workload_flops(wl)
+    run = (setup_attn if attn else setup_mlp)(args, wl, T, stream)
+    step, inp, dev, Y, flops, dt = (run[k] for k in ("step", "inp", "dev", "Y", "flops", "dt"))
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -558,7 +675,7 @@ def main():
         total_k = sum(v[1] for v in kstats.values())
         dom, (dom_launches, dom_ms) = max(kstats.items(), key=lambda kv: kv[1][1])
         launches_total = sum(v[0] for v in kstats.values())
-        dom_flops_per_launch = kernel_flops_per_step(dom, wl) / (dom_launches / args.steps)
+        dom_flops_per_launch = run["kernel_flops"](dom) / (dom_launches / args.steps)
         achieved = dom_flops_per_launch / (dom_ms / dom_launches * 1e-3) / 1e12
         traffic = traffic_for(dom, traffic_key, dom_launches // args.steps) if traffic_key else None
         if dt == "f32":
@@ -567,23 +684,18 @@ def main():
         else:
             bound, peak, peak_src = "tensor", pk["bf16_tflops"], pk["source"]
         line = {
-            "metric": metric_name(wl),
+            "metric": run["metric"],
             "value": tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": dt,
             "data": f"synthetic (seeded torch.randn, cast to {dt})",
-            "tokens_per_s": world * n / (ms * 1e-3),
+            "tokens_per_s": world * run["tokens"] / (ms * 1e-3),
             "pct_of_bf16_peak": 100.0 * tflops / (world * pk["bf16_tflops"]),
             # a sustained (power-capped) peak applies only to a timed region of
             # seconds; a short burst is compared with the burst peak alone
             **({"pct_of_bf16_peak_sustained": 100.0 * tflops / (world * pk["bf16_tflops_sustained"])}
                if long_region else {}),
-            "config": {"workload": wl.name, "n_tokens": n, "d_model": d, "d_ff": f, "P": P,
-                       "act": wl.act, "schedule": sched, "parallelism": f"replicas{world}",
-                       **({"backward": "saved activations" if saved_act else "recompute"}
-                          if wl.backward else {}),
-                       "l2": "inputs larger than L2 (weights 3 x d x f bf16), no flush"
-                       if dt == "bf16" else "inputs fit in L2 (launch-latency bound), no flush"},
+            "config": {**run["config"], "parallelism": f"replicas{world}"},
             "roofline": {"bound": bound, "kernel": dom, "achieved": achieved,
                          "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak,
@@ -603,7 +715,7 @@ def main():
             "clocks": clocks,
         }
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(wl)
+            line["cpu_baseline"] = run["cpu_baseline"]()
         print(json.dumps(line), flush=True)
 
     if dist is not None:

@@ -292,6 +292,66 @@ TSP_API tsp_status_t tsp_mlp_backward_saved(const void* X, const void* W_gate, c
                                             void* workspace, size_t workspace_bytes,
                                             tsp_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * TSP attention: multi-head self-attention under the attention schedule of
+ * "Folding Tensor and Sequence Parallelism for Memory-Efficient Transformer
+ * Training & Inference", Abstract -- every rank holds one sequence shard of
+ * tokens, the ranks iterate over the broadcast parameter shards (groups of
+ * heads), and each reconstructs the whole context through a sequence-wise
+ * key/value exchange.  The head split itself is "Tensor Parallelism:
+ * Splitting the Math", section "Why the column-then-row split -- and what
+ * happens in attention": heads are independent, so W_q, W_k, W_v split by
+ * columns and W_o by rows, with one sum of the partial outputs.
+ *
+ *   Q = X.W_q, K = X.W_k, V = X.W_v                 (head h: columns [128 h, 128 h + 128))
+ *   O_h = softmax(Q_h K_h^T / sqrt(128) + M) V_h    (M = -inf above the diagonal when causal)
+ *   Y = [O_0 | O_1 | ...] . W_o
+ *
+ * Here the P sequence shards (tokens [s n/P, (s+1) n/P)) and the P parameter
+ * shards (heads [w H/P, (w+1) H/P)) are logical.  The queries of sequence
+ * shard s visit the key/value shards in ring order s, s+1, ..., s-1 (mod P),
+ * 128 keys a block, each block merged into a running row maximum, row sum and
+ * weighted value sum in fp32 (tensor memory), so the result is the exact
+ * softmax up to rounding for every P.  With the causal mask the shards after
+ * s hold only future keys and are skipped.  Y_s accumulates the parameter
+ * shards' partial outputs O_{s,w} . W_o[rows of w] in shard order, in fp32
+ * tensor memory, rounded to bf16 once.
+ *
+ * Layout and types: X, Y, Q, K, V, O are [n_tokens][d_model] bf16 row-major,
+ * W_q, W_k, W_v, W_o are [d_model][d_model] bf16 row-major (torch.nn.Linear
+ * stores the transposes).  Head dimension 128: d_model = 128 n_heads.
+ * Q, K, V and the probabilities are rounded to bf16 before their products;
+ * all products accumulate in fp32.
+ *
+ * Requirements: n_tokens > 0, n_tokens % P == 0, n_tokens <= 2^28,
+ * d_model == 128 n_heads, every pointer 16-byte aligned, outputs overlapping
+ * no input.  Errors as for the MLP calls. */
+
+/* The attention core alone: O from Q, K, V (all [n_tokens][d_model] bf16),
+ * sequence shard s's queries over the key/value shards in ring order.
+ * causal != 0 applies the causal mask.  Allocates nothing. */
+TSP_API tsp_status_t tsp_attn_core(const void* Q, const void* K, const void* V, int64_t n_tokens,
+                                   int64_t d_model, int n_heads, int P, int causal, void* O,
+                                   tsp_stream_t stream);
+
+/* Workspace bytes of tsp_attn_forward: Q, K, V and O, [n_tokens][d_model]
+ * bf16 each, 256-byte aligned.  Needs n_heads % P == 0.  No device is
+ * touched. */
+TSP_API tsp_status_t tsp_attn_workspace_size(int64_t n_tokens, int64_t d_model, int n_heads, int P,
+                                             size_t* bytes);
+
+/* The attention block, Y = attention(X) . W_o, under the TSP schedule: the
+ * three projections (every parameter shard's columns for every sequence
+ * shard's tokens, one launch each), the attention core as tsp_attn_core, and
+ * the output projection summing the parameter shards' partial outputs in
+ * order.  Needs n_heads % P == 0 and a workspace of tsp_attn_workspace_size
+ * bytes (256-byte aligned, overlapping no argument). */
+TSP_API tsp_status_t tsp_attn_forward(const void* X, const void* W_q, const void* W_k,
+                                      const void* W_v, const void* W_o, int64_t n_tokens,
+                                      int64_t d_model, int n_heads, int P, int causal, void* Y,
+                                      void* workspace, size_t workspace_bytes,
+                                      tsp_stream_t stream);
+
 /* A static, human-readable name for a status. */
 TSP_API const char* tsp_status_string(tsp_status_t status);
 

@@ -80,6 +80,9 @@ def load(path: str | None = None) -> ctypes.CDLL:
                                                           ctypes.POINTER(ctypes.c_size_t)]
     lib.tsp_mlp_backward_saved.argtypes = [vp, vp, vp, vp, vp, vp, sz, i64, i64, i64, ci, ci, vp,
                                            vp, vp, vp, vp, sz, vp]
+    lib.tsp_attn_core.argtypes = [vp, vp, vp, i64, i64, ci, ci, ci, vp, vp]
+    lib.tsp_attn_workspace_size.argtypes = [i64, i64, ci, ci, ctypes.POINTER(ctypes.c_size_t)]
+    lib.tsp_attn_forward.argtypes = [vp, vp, vp, vp, vp, i64, i64, ci, ci, ci, vp, vp, sz, vp]
     lib.tsp_status_string.argtypes = [ci]
     lib.tsp_status_string.restype = ctypes.c_char_p
     lib.tsp_poll_device_error.argtypes = [vp]
@@ -92,7 +95,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
                  "tsp_mlp_backward_ex", "tsp_mlp_workspace_size", "tsp_poll_device_error",
                  "tsp_trace_enable", "tsp_trace_collect", "tsp_trace_reset",
                  "tsp_selftest_timeout", "tsp_mlp_saved_size", "tsp_mlp_forward_train",
-                 "tsp_mlp_backward_saved_workspace_size", "tsp_mlp_backward_saved"):
+                 "tsp_mlp_backward_saved_workspace_size", "tsp_mlp_backward_saved",
+                 "tsp_attn_core", "tsp_attn_workspace_size", "tsp_attn_forward"):
         getattr(lib, name).restype = ci
     if path is None:
         _lib = lib
@@ -230,6 +234,32 @@ def tsp_mlp_backward_saved(X, W_gate, W_up, W_down, dY, saved, saved_bytes, n_to
     return s
 
 
+def tsp_attn_core(Q, K, V, n_tokens, d_model, n_heads, P, causal, O, stream=None,
+                  check=True) -> int:
+    s = load().tsp_attn_core(_addr(Q), _addr(K), _addr(V), n_tokens, d_model, n_heads, P,
+                             1 if causal else 0, _addr(O), _stream(stream))
+    if check:
+        _check(s, "tsp_attn_core")
+    return s
+
+
+def tsp_attn_workspace_size(n_tokens, d_model, n_heads, P) -> int:
+    out = ctypes.c_size_t(0)
+    s = load().tsp_attn_workspace_size(n_tokens, d_model, n_heads, P, ctypes.byref(out))
+    _check(s, "tsp_attn_workspace_size")
+    return int(out.value)
+
+
+def tsp_attn_forward(X, W_q, W_k, W_v, W_o, n_tokens, d_model, n_heads, P, causal, Y, workspace,
+                     workspace_bytes, stream=None, check=True) -> int:
+    s = load().tsp_attn_forward(_addr(X), _addr(W_q), _addr(W_k), _addr(W_v), _addr(W_o),
+                                n_tokens, d_model, n_heads, P, 1 if causal else 0, _addr(Y),
+                                _addr(workspace), workspace_bytes, _stream(stream))
+    if check:
+        _check(s, "tsp_attn_forward")
+    return s
+
+
 def tsp_status_string(status: int) -> str:
     return load().tsp_status_string(int(status)).decode()
 
@@ -342,3 +372,26 @@ def mlp_backward_saved(X, W_gate, W_up, W_down, dY, saved, P: int, act: str, wor
     tsp_mlp_backward_saved(X, W_gate, W_up, W_down, dY, saved, _nbytes(saved), n, d, f, P, act, dX,
                            dWg, dWu, dWd, ws, need, stream)
     return dX, dWg, dWu, dWd
+
+
+def attn_core(Q, K, V, n_heads: int, P: int, causal: bool, out=None, stream=None):
+    """O = attention(Q, K, V) through tsp_attn_core (bf16 [n, d] each)."""
+    import torch
+    n, d = Q.shape
+    O = out if out is not None else torch.empty((n, d), dtype=torch.bfloat16, device=Q.device)
+    tsp_attn_core(Q, K, V, n, d, n_heads, P, causal, O, stream)
+    return O
+
+
+def attn_forward(X, W_q, W_k, W_v, W_o, n_heads: int, P: int, causal: bool, workspace=None,
+                 out=None, stream=None):
+    """Y = attention block (X) under the TSP schedule through tsp_attn_forward;
+    allocates Y and the workspace with torch unless given."""
+    import torch
+    n, d = X.shape
+    Y = out if out is not None else torch.empty((n, d), dtype=torch.bfloat16, device=X.device)
+    need = tsp_attn_workspace_size(n, d, n_heads, P)
+    ws = workspace if workspace is not None else torch.empty(need, dtype=torch.uint8,
+                                                              device=X.device)
+    tsp_attn_forward(X, W_q, W_k, W_v, W_o, n, d, n_heads, P, causal, Y, ws, _nbytes(ws), stream)
+    return Y

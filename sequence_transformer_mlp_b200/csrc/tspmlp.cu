@@ -13,12 +13,14 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
 #include <vector>
 
 #include "../../include/tspmlp.h"
+#include "attn.cuh"
 #include "bwd_pair.cuh"
 #include "train_pair.cuh"
 #include "grad_pair.cuh"
@@ -169,7 +171,8 @@ void trace_end(cudaStream_t st, TraceRec* rec) {
 // Paired launch: clusters of two CTAs (cta_group::2 tiles), as many pairs as
 // can be resident at once, each walking the tile list persistently.
 template <class R>
-tsp_status_t launch_pair(const typename R::Params& p, cudaStream_t st, int dev, int sms) {
+tsp_status_t launch_pair(const typename R::Params& p, cudaStream_t st, int dev, int sms,
+                         const char* trace_name = nullptr) {
     const int tiles = R::num_tiles(p);
     if (tiles <= 0) return TSP_OK;
     constexpr int smem = pair_smem_bytes<R>();
@@ -213,7 +216,7 @@ tsp_status_t launch_pair(const typename R::Params& p, cudaStream_t st, int dev, 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     TraceRec rec;
-    const bool traced = trace_begin(st, &rec, R::kName);
+    const bool traced = trace_begin(st, &rec, trace_name ? trace_name : R::kName);
     const cudaError_t e = cudaLaunchKernelEx(&cfg, umma_pair_pipeline_kernel<R>, p);
     if (traced) trace_end(st, &rec);
     return e == cudaSuccess ? TSP_OK : TSP_ERR_CUDA;
@@ -1204,6 +1207,83 @@ tsp_status_t backward_bf16(const void* X, const void* Wg, const void* Wu, const 
     return TSP_OK;
 }
 
+
+// ---------------------------------------------------------------------------
+// TSP attention ("Folding Tensor and Sequence Parallelism ...", Abstract: the
+// attention schedule).  Head dimension 128.
+
+constexpr int kAttnHeadDim = 128;
+
+tsp_status_t validate_attn_shape(int64_t n, int64_t d, int heads, int P) {
+    if (n <= 0 || d <= 0 || heads <= 0 || P <= 0) return TSP_ERR_INVALID_ARG;
+    if (n > (int64_t(1) << 28) || d > 65536 || P > 4096) return TSP_ERR_UNSUPPORTED_SHAPE;
+    if (d != static_cast<int64_t>(heads) * kAttnHeadDim) return TSP_ERR_UNSUPPORTED_SHAPE;
+    if (n % P != 0) return TSP_ERR_UNSUPPORTED_SHAPE;
+    return TSP_OK;
+}
+
+// C[m][nout] = A[m][k] . B[k][nout], bf16 out, fp32 accumulate in tensor
+// memory: the paired down-projection recipe with one K segment, stored direct.
+tsp_status_t gemm_bf16(const void* A, const void* B, int64_t m, int64_t k, int64_t nout, void* Cm,
+                       cudaStream_t st, int dev, int sms, const char* trace_name) {
+    using K2 = DownAccum<true, 1>;
+    typename K2::Params p2;
+    std::memset(&p2, 0, sizeof(p2));
+    if (!tmap_bf16(&p2.tmA0, A, k, m, k, 64, 128, SW128) ||
+        !tmap_bf16(&p2.tmB0, B, nout, k, nout, 64, 128, SW128))
+        return TSP_ERR_CUDA;
+    p2.g = seg_all_rows(m, 1, k, 0);
+    p2.kdim = static_cast<int>(k);
+    p2.n_out = static_cast<int>(nout);
+    p2.mode = 3;
+    p2.rot_P = 0;
+    p2.acc = nullptr;
+    p2.out = static_cast<__nv_bfloat16*>(Cm);
+    p2.ldo = nout;
+    return launch_pair<DownAccumPair<true, 1, 256>>(p2, st, dev, sms, trace_name);
+}
+
+tsp_status_t launch_attn_core(const void* Q, const void* K, const void* V, int64_t n, int64_t d,
+                              int heads, int P, int causal, void* O, cudaStream_t st, int dev,
+                              int sms) {
+    AttnParams p;
+    std::memset(&p, 0, sizeof(p));
+    if (!tmap_bf16(&p.tmQ, Q, d, n, d, 64, 128, SW128) ||
+        !tmap_bf16(&p.tmK, K, d, n, d, 64, 128, SW128) ||
+        !tmap_bf16(&p.tmV, V, d, n, d, 64, 128, SW128))
+        return TSP_ERR_CUDA;
+    p.O = static_cast<__nv_bfloat16*>(O);
+    p.ldo = d;
+    p.n = static_cast<int>(n);
+    p.heads = heads;
+    p.P = P;
+    p.ns = static_cast<int>(n / P);
+    p.nb = (p.ns + 127) / 128;
+    p.npr = (p.ns + 255) / 256;
+    p.causal = causal ? 1 : 0;
+    p.items = heads * P * p.npr;
+    p.sl2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(kAttnHeadDim)));
+    constexpr int smem = AttnCore::kSmemBytes;
+    static_assert(smem <= 232448, "attention core exceeds 227 KB of shared memory");
+    static bool attr_set[kMaxDevices] = {};
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!attr_set[dev]) {
+            if (cudaFuncSetAttribute(attn_core_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     smem) != cudaSuccess)
+                return TSP_ERR_CUDA;
+            attr_set[dev] = true;
+        }
+    }
+    const int grid = std::min(p.items, sms);
+    TraceRec rec;
+    const bool traced = trace_begin(st, &rec, causal ? "attn_core_causal" : "attn_core");
+    attn_core_kernel<<<grid, AttnCore::kThreads, smem, st>>>(p);
+    const cudaError_t e = cudaGetLastError();
+    if (traced) trace_end(st, &rec);
+    return e == cudaSuccess ? TSP_OK : TSP_ERR_CUDA;
+}
+
 }  // namespace
 }  // namespace tspmlp
 
@@ -1433,6 +1513,68 @@ tsp_status_t tsp_mlp_backward_saved(const void* X, const void* Wg, const void* W
                                 di.sms, &sv);
     return backward_bf16<0>(X, Wg, Wu, Wd, dY, n, d, f, P, pl, dX, dWg, dWu, dWd, ws, st, dev,
                             di.sms, &sv);
+}
+
+tsp_status_t tsp_attn_core(const void* Q, const void* K, const void* V, int64_t n, int64_t d,
+                           int n_heads, int P, int causal, void* O, tsp_stream_t stream) {
+    TSP_TRY(validate_attn_shape(n, d, n_heads, P));
+    if (!Q || !K || !V || !O) return TSP_ERR_INVALID_ARG;
+    const size_t b = n * d * 2;
+    if (overlaps(O, b, Q, b) || overlaps(O, b, K, b) || overlaps(O, b, V, b))
+        return TSP_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
+        return TSP_ERR_UNSUPPORTED_SHAPE;
+    int dev = 0;
+    DevInfo di;
+    TSP_TRY(current_device(&dev, &di));
+    return launch_attn_core(Q, K, V, n, d, n_heads, P, causal, O,
+                            reinterpret_cast<cudaStream_t>(stream), dev, di.sms);
+}
+
+tsp_status_t tsp_attn_workspace_size(int64_t n, int64_t d, int n_heads, int P, size_t* bytes) {
+    if (!bytes) return TSP_ERR_INVALID_ARG;
+    TSP_TRY(validate_attn_shape(n, d, n_heads, P));
+    if (n_heads % P != 0) return TSP_ERR_UNSUPPORTED_SHAPE;
+    *bytes = 4 * align256(static_cast<size_t>(n) * d * 2);
+    return TSP_OK;
+}
+
+tsp_status_t tsp_attn_forward(const void* X, const void* Wq, const void* Wk, const void* Wv,
+                              const void* Wo, int64_t n, int64_t d, int n_heads, int P, int causal,
+                              void* Y, void* ws, size_t ws_bytes, tsp_stream_t stream) {
+    TSP_TRY(validate_attn_shape(n, d, n_heads, P));
+    if (n_heads % P != 0) return TSP_ERR_UNSUPPORTED_SHAPE;
+    if (!X || !Wq || !Wk || !Wv || !Wo || !Y) return TSP_ERR_INVALID_ARG;
+    const void* ins[5] = {X, Wq, Wk, Wv, Wo};
+    for (const void* q : ins)
+        if (!aligned16(q)) return TSP_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(Y)) return TSP_ERR_UNSUPPORTED_SHAPE;
+    const size_t xb = n * d * 2, wb = d * d * 2;
+    const size_t isz[5] = {xb, wb, wb, wb, wb};
+    for (int i = 0; i < 5; ++i)
+        if (overlaps(Y, xb, ins[i], isz[i])) return TSP_ERR_INVALID_ARG;
+    const size_t one = align256(xb), need = 4 * one;
+    if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) return TSP_ERR_WORKSPACE;
+    for (int i = 0; i < 5; ++i)
+        if (overlaps(ws, need, ins[i], isz[i])) return TSP_ERR_INVALID_ARG;
+    if (overlaps(ws, need, Y, xb)) return TSP_ERR_INVALID_ARG;
+    int dev = 0;
+    DevInfo di;
+    TSP_TRY(current_device(&dev, &di));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    char* w = static_cast<char*>(ws);
+    void *Q = w, *K = w + one, *V = w + 2 * one, *O = w + 3 * one;
+    // every parameter shard's columns of W_q, W_k, W_v, for every sequence
+    // shard's tokens: the projections of all (shard, shard) pairs in one
+    // launch each (no sum crosses shards)
+    TSP_TRY(gemm_bf16(X, Wq, n, d, d, Q, st, dev, di.sms, "attn_proj"));
+    TSP_TRY(gemm_bf16(X, Wk, n, d, d, K, st, dev, di.sms, "attn_proj"));
+    TSP_TRY(gemm_bf16(X, Wv, n, d, d, V, st, dev, di.sms, "attn_proj"));
+    // each sequence shard's queries over the key/value shards in ring order
+    TSP_TRY(launch_attn_core(Q, K, V, n, d, n_heads, P, causal, O, st, dev, di.sms));
+    // Y_s = sum over parameter shards w (in order) of O_{s,w} . W_o[rows of w]:
+    // the K loop runs over the head groups in order, summing in tensor memory
+    return gemm_bf16(O, Wo, n, d, d, Y, st, dev, di.sms, "attn_out_proj");
 }
 
 tsp_status_t tsp_trace_enable(int enable) {

@@ -214,3 +214,35 @@ def test_training_pair_rejects_bad_buffers(lib):
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(ImportError):
         T.load(str(tmp_path / "nope.so"))
+
+
+def test_attention_workspace_and_shape_rules(lib):
+    # Q, K, V, O: [n][d] bf16 each, 256-byte aligned
+    assert T.tsp_attn_workspace_size(32768, 4096, 32, 8) == 4 * 32768 * 4096 * 2
+    assert T.tsp_attn_workspace_size(3, 128, 1, 1) == 4 * _a256(3 * 128 * 2)
+    out = ctypes.c_size_t(0)
+    # head dimension 128 only; tokens a multiple of P; heads a multiple of P
+    assert lib.tsp_attn_workspace_size(64, 4096, 64, 8, ctypes.byref(out)) == 2
+    assert lib.tsp_attn_workspace_size(100, 1024, 8, 8, ctypes.byref(out)) == 2
+    assert lib.tsp_attn_workspace_size(96, 1024, 8, 3, ctypes.byref(out)) == 2
+    assert lib.tsp_attn_workspace_size(0, 1024, 8, 8, ctypes.byref(out)) == 1
+    assert lib.tsp_attn_workspace_size(64, 1024, 8, 8, None) == 1
+
+
+def test_attention_bad_arguments_are_rejected_before_any_device_call(lib):
+    X, Wq, Wk, Wv, Wo, Y, W = (k << 32 for k in range(1, 8))
+    n, d, h, P = 256, 256, 2, 2
+    ws = T.tsp_attn_workspace_size(n, d, h, P)
+    fw = T.tsp_attn_forward
+    assert fw(None, Wq, Wk, Wv, Wo, n, d, h, P, True, Y, W, ws, stream=0, check=False) == 1
+    assert fw(X, Wq, Wk, Wv, Wo, n, d, h, P, True, X + 64, W, ws, stream=0, check=False) == 1
+    assert fw(X + 2, Wq, Wk, Wv, Wo, n, d, h, P, True, Y, W, ws, stream=0, check=False) == 2
+    assert fw(X, Wq, Wk, Wv, Wo, n, d, h, P, True, Y, W, ws - 1, stream=0, check=False) == 6
+    assert fw(X, Wq, Wk, Wv, Wo, n, d, h, P, True, Y, W + 16, ws, stream=0, check=False) == 6
+    assert fw(X, Wq, Wk, Wv, Wo, n, d, h, P, True, Y, X, ws, stream=0, check=False) == 1
+    assert fw(X, Wq, Wk, Wv, Wo, n, d, h, 4, True, Y, W, ws, stream=0, check=False) == 2
+    core = T.tsp_attn_core
+    assert core(X, Wq, Wk, n, d, h, P, False, None, stream=0, check=False) == 1
+    assert core(X, Wq, Wk, n, d, h, P, False, Wq + 512, stream=0, check=False) == 1
+    assert core(X, Wq, Wk, n, 192, h, P, False, Y, stream=0, check=False) == 2
+    assert core(X, Wq, Wk, 255, d, h, P, False, Y, stream=0, check=False) == 2

@@ -53,3 +53,14 @@ def test_cpu_baseline_reports_the_whole_step():
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] > 0
     assert cb["extrapolated_full_step_s"] > 0
     assert "input gradient" in cb["sample"] and "weight gradients" in cb["sample"]
+
+
+def test_attention_cpu_baseline_extrapolates_from_two_row_counts():
+    from workloads import AttnWorkload, make_attn_inputs
+    wl = AttnWorkload("tiny_attn", 64, 256, 2, 2, True, seed=3, w_std=0.05)
+    parts = bench.attn_oracle_sample(wl, make_attn_inputs(wl), 8)
+    assert parts["extrapolated_full_step_s"] >= parts["fixed_s"] >= 0
+    assert abs(parts["extrapolated_full_step_s"]
+               - (parts["fixed_s"] + parts["per_row_s"] * 64)) < 1e-12
+    cb = bench.attn_cpu_baseline(wl, rows=8)
+    assert cb["kind"] == "oracle" and cb["value"] > 0

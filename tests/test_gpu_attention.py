@@ -1,0 +1,158 @@
+"""GPU parity of the TSP attention schedule against the fp64 oracle, through the
+C ABI (tsp_attn_core, tsp_attn_forward).
+
+Tolerance: the bf16 bar of the MLP tests -- max|O - Oref| <= 1e-2 max|Oref|
+and relative Frobenius error <= 5e-3.  The oracle sees the exact bf16 inputs
+widened to fp64; the kernel rounds the probabilities (and, in the block, Q, K,
+V and O) to bf16 before their products and accumulates in fp32.
+
+The core is compared element by element at small and ragged shapes (several
+key blocks and query tiles, sequence shards that are not a multiple of 128
+tokens, one-token shards, both masks, a key scale that grows along the ring so
+that the running maximum moves and O is rescaled).  The full-size workload is
+compared on sampled query rows: a row of Y depends on its own query and on
+every key and value, all of which the oracle computes.
+"""
+import numpy as np
+import pytest
+import torch
+
+import sequence_transformer_mlp_b200 as T
+from oracle import attention as OA
+from workloads import AttnWorkload, TSP_ATTN, cover_rows, make_attn_inputs, make_qkv
+
+pytestmark = pytest.mark.gpu
+
+
+def check(got, ref, what):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert got.shape == ref.shape, what
+    assert np.isfinite(got).all(), f"{what}: non-finite output"
+    mx = float(np.abs(ref).max())
+    err = float(np.abs(got - ref).max())
+    fro = float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300))
+    print(f"PARITY {what} max_rel={err / mx:.3e} fro={fro:.3e}")
+    assert err <= 1e-2 * mx, f"{what}: max|d|/max|ref| = {err / mx:.3e}"
+    assert fro <= 5e-3, f"{what}: rel Frobenius {fro:.3e}"
+
+
+def np64(t):
+    return t.float().cpu().double().numpy()
+
+
+def gpu_core(qkv, heads, P, causal):
+    d = {k: v.cuda() for k, v in qkv.items()}
+    O = T.attn_core(d["Q"], d["K"], d["V"], heads, P, causal)
+    torch.cuda.synchronize()
+    assert T.tsp_poll_device_error() == T.TSP_OK
+    return O
+
+
+CORE_CASES = [
+    # n, heads, P -- one query pair; several key blocks; shards of 150, 125 and
+    # 100 tokens (ragged key blocks and query tiles); 3 and 5 shards of 128
+    (256, 1, 1),
+    (512, 2, 2),
+    (300, 1, 2),
+    (1000, 2, 8),
+    (384, 1, 3),
+    (640, 2, 5),
+    (800, 1, 8),
+]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("n,heads,P", CORE_CASES)
+def test_core_small_shapes(n, heads, P, causal):
+    qkv = make_qkv(n, 128 * heads, seed=n + heads + P)
+    O = gpu_core(qkv, heads, P, causal)
+    ref = OA.attention_core(qkv["Q"], qkv["K"], qkv["V"], heads, causal)
+    check(np64(O), ref, f"core n={n} h={heads} P={P} causal={causal}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("n,P", [(1, 1), (8, 8), (24, 8), (129, 1)])
+def test_core_degenerate_shapes(n, P, causal):
+    """One token; one-token and three-token sequence shards; one key past a block."""
+    qkv = make_qkv(n, 128, seed=40 + n)
+    O = gpu_core(qkv, 1, P, causal)
+    ref = OA.attention_core(qkv["Q"], qkv["K"], qkv["V"], 1, causal)
+    check(np64(O), ref, f"core degenerate n={n} P={P}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_core_peaked_scores_and_growing_maximum(causal):
+    """Scores with std 4, and keys scaled up along the sequence so that every
+    sequence shard meets larger scores later in its ring: the running maximum
+    moves by more than 2^8 and O is rescaled in tensor memory."""
+    n, heads, P = 1024, 2, 4
+    qkv = make_qkv(n, 128 * heads, seed=77, std=2.0)
+    grow = torch.linspace(0.5, 3.0, n).unsqueeze(1)
+    qkv["K"] = (qkv["K"].float() * grow).to(torch.bfloat16).contiguous()
+    O = gpu_core(qkv, heads, P, causal)
+    ref = OA.attention_core(qkv["Q"], qkv["K"], qkv["V"], heads, causal)
+    check(np64(O), ref, f"core peaked causal={causal}")
+    ref_tsp = OA.attention_core_tsp(qkv["Q"], qkv["K"], qkv["V"], heads, P, causal)
+    check(np64(O), ref_tsp, "core peaked vs the ring-ordered oracle")
+
+
+def test_core_independent_of_P():
+    qkv = make_qkv(768, 256, seed=5)
+    ref = OA.attention_core(qkv["Q"], qkv["K"], qkv["V"], 2, True)
+    for P in (1, 2, 3, 4, 6):
+        check(np64(gpu_core(qkv, 2, P, True)), ref, f"core P={P}")
+
+
+def test_core_run_to_run_bitwise_deterministic():
+    qkv = make_qkv(1000, 256, seed=6)
+    a = gpu_core(qkv, 2, 8, True)
+    b = gpu_core(qkv, 2, 8, True)
+    assert torch.equal(a, b)
+
+
+# ---------------------------------------------------------------------------- the block
+
+
+BLOCK_CASES = [
+    # n, d, heads, P, causal
+    (512, 256, 2, 2, True),
+    (512, 256, 2, 2, False),
+    (768, 512, 4, 4, True),
+    (1000, 1024, 8, 8, True),
+    (600, 384, 3, 3, False),
+]
+
+
+@pytest.mark.parametrize("n,d,heads,P,causal", BLOCK_CASES)
+def test_block_small_shapes(n, d, heads, P, causal):
+    wl = AttnWorkload("attn_small", n, d, heads, P, causal, seed=n + d, w_std=0.05)
+    inp = make_attn_inputs(wl)
+    dev = {k: v.cuda() for k, v in inp.items()}
+    Y = T.attn_forward(dev["X"], dev["Wq"], dev["Wk"], dev["Wv"], dev["Wo"], heads, P, causal)
+    torch.cuda.synchronize()
+    assert T.tsp_poll_device_error() == T.TSP_OK
+    ref = OA.attention_tsp(inp["X"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wo"], heads, P, causal)
+    check(np64(Y), ref, f"block n={n} d={d} P={P} causal={causal}")
+
+
+def test_block_long_context_sampled_rows():
+    """The TSP attention workload (32768 tokens in 8 sequence shards of 4096,
+    32 heads of 128 in 8 parameter shards, causal), in the launch configuration
+    the benchmark times.  Rows: one seeded row in each of the 128 blocks of 256
+    tokens (every query-tile pair of every sequence shard, so every work item's
+    ring start and diagonal position), plus each sequence shard's first and
+    last row."""
+    wl = TSP_ATTN
+    inp = make_attn_inputs(wl)
+    dev = {k: v.cuda() for k, v in inp.items()}
+    Y = T.attn_forward(dev["X"], dev["Wq"], dev["Wk"], dev["Wv"], dev["Wo"], wl.heads, wl.P,
+                       wl.causal)
+    torch.cuda.synchronize()
+    assert T.tsp_poll_device_error() == T.TSP_OK
+    ns = wl.n // wl.P
+    rows = cover_rows(wl.n, 256, wl.seed, groups=[(s * ns, (s + 1) * ns) for s in range(wl.P)])
+    assert len(rows) >= 128
+    ref = OA.attention_forward(inp["X"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wo"], wl.heads,
+                               wl.causal, rows=rows)
+    check(np64(Y[rows]), ref, f"{wl.name} sampled rows")
