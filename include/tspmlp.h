@@ -42,7 +42,8 @@
  * returns a status and touches nothing.  Kernels bound every wait on the GPU
  * (about two seconds); a wait that runs out sets the device error word and the
  * kernel returns early, so a later tsp_poll_device_error() reports
- * TSP_ERR_TIMEOUT instead of hanging.  All calls are asynchronous on `stream`.
+ * TSP_ERR_TIMEOUT instead of hanging (TSP_ERR_RANGE: see TSP attention).  All
+ * calls are asynchronous on `stream`.
  */
 #ifndef TSPMLP_H
 #define TSPMLP_H
@@ -72,7 +73,10 @@ typedef enum {
     TSP_ERR_CUDA = 4,              /* a CUDA runtime call or launch failed */
     TSP_ERR_TIMEOUT = 5,           /* a bounded device-side wait ran out */
     TSP_ERR_WORKSPACE = 6,         /* workspace NULL or smaller than tsp_mlp_workspace_size */
-    TSP_ERR_SCRATCH_LIMIT = 7      /* needs more scratch than tsp_mlp_forward_noalloc holds */
+    TSP_ERR_SCRATCH_LIMIT = 7,     /* needs more scratch than tsp_mlp_forward_noalloc holds */
+    TSP_ERR_RANGE = 8              /* reported by tsp_poll_device_error: an fp16 intermediate
+                                    * (tsp_attn_forward's Q or K) exceeded 65504 in magnitude
+                                    * and was saturated */
 } tsp_status_t;
 
 typedef enum {
@@ -317,11 +321,15 @@ TSP_API tsp_status_t tsp_mlp_backward_saved(const void* X, const void* W_gate, c
  * shards' partial outputs O_{s,w} . W_o[rows of w] in shard order, in fp32
  * tensor memory, rounded to bf16 once.
  *
- * Layout and types: X, Y, Q, K, V, O are [n_tokens][d_model] bf16 row-major,
+ * Layout and types: X, Y, Q, K, V, O are [n_tokens][d_model] row-major,
  * W_q, W_k, W_v, W_o are [d_model][d_model] bf16 row-major (torch.nn.Linear
  * stores the transposes).  Head dimension 128: d_model = 128 n_heads.
- * Q, K, V and the probabilities are rounded to bf16 before their products;
- * all products accumulate in fp32.
+ * X, Y, V, O and the weights are bf16.  tsp_attn_core takes bf16 Q and K;
+ * tsp_attn_forward keeps its own Q and K in fp16 (three more mantissa bits
+ * where the scores' rounding matters most): a projected value above 65504 in
+ * magnitude saturates and the next tsp_poll_device_error() returns
+ * TSP_ERR_RANGE.  The probabilities are rounded to bf16 before P.V; all
+ * products accumulate in fp32.
  *
  * Requirements: n_tokens > 0, n_tokens % P == 0, n_tokens <= 2^28,
  * d_model == 128 n_heads, every pointer 16-byte aligned, outputs overlapping
@@ -334,8 +342,8 @@ TSP_API tsp_status_t tsp_attn_core(const void* Q, const void* K, const void* V, 
                                    int64_t d_model, int n_heads, int P, int causal, void* O,
                                    tsp_stream_t stream);
 
-/* Workspace bytes of tsp_attn_forward: Q, K, V and O, [n_tokens][d_model]
- * bf16 each, 256-byte aligned.  Needs n_heads % P == 0.  No device is
+/* Workspace bytes of tsp_attn_forward: Q, K (fp16), V and O (bf16),
+ * [n_tokens][d_model] each, 256-byte aligned.  Needs n_heads % P == 0.  No device is
  * touched. */
 TSP_API tsp_status_t tsp_attn_workspace_size(int64_t n_tokens, int64_t d_model, int n_heads, int P,
                                              size_t* bytes);
@@ -388,8 +396,9 @@ TSP_API tsp_status_t tsp_trace_reset(void);
 TSP_API tsp_status_t tsp_selftest_timeout(int mode, tsp_stream_t stream);
 
 /* Synchronises `stream`, then reads and clears the current device's error
- * word: TSP_OK, TSP_ERR_TIMEOUT if a kernel gave up waiting, TSP_ERR_CUDA if
- * the stream reported an error. */
+ * word: TSP_OK, TSP_ERR_TIMEOUT if a kernel gave up waiting, TSP_ERR_RANGE if
+ * an fp16 intermediate saturated (and no wait ran out), TSP_ERR_CUDA if the
+ * stream reported an error. */
 TSP_API tsp_status_t tsp_poll_device_error(tsp_stream_t stream);
 
 #ifdef __cplusplus

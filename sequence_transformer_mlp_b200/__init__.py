@@ -31,6 +31,7 @@ STATUS_NAMES = {
     5: "TSP_ERR_TIMEOUT",
     6: "TSP_ERR_WORKSPACE",
     7: "TSP_ERR_SCRATCH_LIMIT",
+    8: "TSP_ERR_RANGE",
 }
 NOALLOC_SCRATCH_BYTES = 32 << 20
 ACT = {"gelu": 0, "swiglu": 1}

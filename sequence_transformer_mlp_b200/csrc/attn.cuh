@@ -69,7 +69,8 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 }
 
 struct AttnParams {
-    CUtensorMap tmQ, tmK, tmV;  // [n][heads * 128] bf16, box {64, 128}, 128-byte swizzle
+    CUtensorMap tmQ, tmK, tmV;  // [n][heads * 128] (Q, K bf16 or fp16; V bf16), box {64, 128},
+                                // 128-byte swizzle
     __nv_bfloat16* O;           // [n][ldo] bf16
     long long ldo;
     int n;       // tokens
@@ -99,7 +100,10 @@ struct AttnCore {
     static constexpr int kQOff = 0, kPOff = 2 * kTileBytes, kKVOff = 4 * kTileBytes;
     static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
     static constexpr int kSmemBytes = kBarOff + 256 + 1024;
-    static constexpr uint32_t kIdescS = make_idesc_bf16(128, 128, false, false);
+    // Q K^T in fp16 (the block's projections store Q and K as fp16: three more
+    // mantissa bits than bf16 where the scores' rounding matters most) or bf16
+    static constexpr uint32_t kIdescSf16 = make_idesc_f16(128, 128, false, false);
+    static constexpr uint32_t kIdescSbf16 = make_idesc_bf16(128, 128, false, false);
     static constexpr uint32_t kIdescPV = make_idesc_bf16(128, 128, false, true);
     // the running max is moved (and O rescaled) only when a block's max
     // exceeds it by more than this many powers of two
@@ -153,9 +157,11 @@ struct AttnCore {
     }
 };
 
+template <bool QK_F16>
 __global__ void __launch_bounds__(AttnCore::kThreads, 1)
     attn_core_kernel(const __grid_constant__ AttnParams p) {
     using C = AttnCore;
+    constexpr uint32_t kIdescS = QK_F16 ? C::kIdescSf16 : C::kIdescSbf16;
     constexpr int S = C::kStages;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -286,7 +292,7 @@ __global__ void __launch_bounds__(AttnCore::kThreads, 1)
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * 16384 + 32 * (kk & 3);
                     umma_bf16(tmem + 256 + 128 * a, make_smem_desc(qa + off, 16, 1024, kLayoutSW128),
-                              make_smem_desc(kb + off, 16, 1024, kLayoutSW128), C::kIdescS,
+                              make_smem_desc(kb + off, 16, 1024, kLayoutSW128), kIdescS,
                               kk != 0 ? 1u : 0u);
                 }
                 umma_commit(s_full(a));

@@ -11,7 +11,10 @@ namespace tspmlp {
 // Device-side error word (one per device; the library is one translation
 // unit).  Bit values below; the host reads and clears it in
 // tsp_poll_device_error().
-enum : uint32_t { kDevErrTimeout = 1u };
+enum : uint32_t {
+    kDevErrTimeout = 1u,  // a bounded wait ran out
+    kDevErrRange = 2u     // a value left the range of an fp16 intermediate
+};
 __device__ uint32_t g_device_error = 0;
 
 // A bounded wait gives up after this many nanoseconds of %globaltimer.
@@ -325,6 +328,13 @@ __host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, bool a_mn, 
            | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
 }
 
+// The same for kind::f16 with fp16 A and B (fp32 D).
+__host__ __device__ constexpr uint32_t make_idesc_f16(int M, int N, bool a_mn, bool b_mn) {
+    return (1u << 4)                                  // D format: f32
+           | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16)
+           | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
 // ---------------------------------------------------------------------------
 // small numeric helpers
 
@@ -337,6 +347,14 @@ __device__ __forceinline__ float bf16hi_to_f32(uint32_t v) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+    return r;
+}
+
+// Two floats -> packed fp16x2 (round to nearest even; magnitudes above the
+// largest finite fp16 become +-65504, not infinity); `a` in the low half.
+__device__ __forceinline__ uint32_t pack_f16x2_sat(float a, float b) {
+    uint32_t r;
+    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
     return r;
 }
 

@@ -203,7 +203,8 @@ struct FwdHidden {
 //   out[rows][0..n_out) (+)= sum over K-segments of A_seg . B_seg
 // A is K-major (hidden activations, [rows][kdim]); B is MN-major (W_down
 // [f][d], forward) or K-major (W_gate / W_up [d][f], input gradient).
-// Modes: 0 store fp32, 1 add into fp32, 2 bf16(acc + tile) to out, 3 bf16(tile).
+// Modes: 0 store fp32, 1 add into fp32, 2 bf16(acc + tile) to out, 3 bf16(tile),
+// 4 fp16(tile) to out (magnitudes above 65504 saturate and raise kDevErrRange).
 // This struct holds the launch parameters and the per-row epilogue; the
 // paired kernel (DownAccumPair in pipeline2.cuh) does the loads and MMAs.
 template <bool B_MN, int NSEG>
@@ -265,6 +266,17 @@ struct DownAccum {
                     for (int i = 0; i < 32; ++i)
                         if (i < valid) a[i] += __uint_as_float(v[i]);
                 }
+            } else if (p.mode == 4) {
+                uint32_t pk[16];
+                bool big = false;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float x0 = __uint_as_float(v[2 * i]), x1 = __uint_as_float(v[2 * i + 1]);
+                    big |= fabsf(x0) > 65504.f || fabsf(x1) > 65504.f;
+                    pk[i] = pack_f16x2_sat(x0, x1);
+                }
+                if (big) atomicOr(&g_device_error, kDevErrRange);
+                store_bf16x32(p.out + row * p.ldo + c0, pk, valid);  // 16-bit words, any format
             } else {
                 uint32_t pk[16];
                 if (p.mode == 2) {

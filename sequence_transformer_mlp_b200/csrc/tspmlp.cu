@@ -126,6 +126,20 @@ bool tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
 
 constexpr CUtensorMapSwizzle SW128 = CU_TENSOR_MAP_SWIZZLE_128B;
 
+// The same for an fp16 matrix.
+bool tmap_f16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t pitch,
+              uint32_t box_in, uint32_t box_out, CUtensorMapSwizzle sw) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {pitch * 2};
+    cuuint32_t box[2] = {box_in, box_out};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+               es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ---------------------------------------------------------------------------
 // tracing: CUDA events around each launch, on the launching stream
 
@@ -1222,10 +1236,12 @@ tsp_status_t validate_attn_shape(int64_t n, int64_t d, int heads, int P) {
     return TSP_OK;
 }
 
-// C[m][nout] = A[m][k] . B[k][nout], bf16 out, fp32 accumulate in tensor
-// memory: the paired down-projection recipe with one K segment, stored direct.
+// C[m][nout] = A[m][k] . B[k][nout] (bf16 A, B), fp32 accumulate in tensor
+// memory: the paired down-projection recipe with one K segment, stored direct
+// as bf16 (out_f16 false) or fp16 (true; magnitudes above 65504 saturate and
+// raise the range bit of the device error word).
 tsp_status_t gemm_bf16(const void* A, const void* B, int64_t m, int64_t k, int64_t nout, void* Cm,
-                       cudaStream_t st, int dev, int sms, const char* trace_name) {
+                       bool out_f16, cudaStream_t st, int dev, int sms, const char* trace_name) {
     using K2 = DownAccum<true, 1>;
     typename K2::Params p2;
     std::memset(&p2, 0, sizeof(p2));
@@ -1235,7 +1251,7 @@ tsp_status_t gemm_bf16(const void* A, const void* B, int64_t m, int64_t k, int64
     p2.g = seg_all_rows(m, 1, k, 0);
     p2.kdim = static_cast<int>(k);
     p2.n_out = static_cast<int>(nout);
-    p2.mode = 3;
+    p2.mode = out_f16 ? 4 : 3;
     p2.rot_P = 0;
     p2.acc = nullptr;
     p2.out = static_cast<__nv_bfloat16*>(Cm);
@@ -1243,13 +1259,15 @@ tsp_status_t gemm_bf16(const void* A, const void* B, int64_t m, int64_t k, int64
     return launch_pair<DownAccumPair<true, 1, 256>>(p2, st, dev, sms, trace_name);
 }
 
+// qk_f16: Q and K are fp16 (the block's own projections), else bf16.
 tsp_status_t launch_attn_core(const void* Q, const void* K, const void* V, int64_t n, int64_t d,
-                              int heads, int P, int causal, void* O, cudaStream_t st, int dev,
-                              int sms) {
+                              int heads, int P, int causal, bool qk_f16, void* O, cudaStream_t st,
+                              int dev, int sms) {
     AttnParams p;
     std::memset(&p, 0, sizeof(p));
-    if (!tmap_bf16(&p.tmQ, Q, d, n, d, 64, 128, SW128) ||
-        !tmap_bf16(&p.tmK, K, d, n, d, 64, 128, SW128) ||
+    auto tmap_qk = qk_f16 ? tmap_f16 : tmap_bf16;
+    if (!tmap_qk(&p.tmQ, Q, d, n, d, 64, 128, SW128) ||
+        !tmap_qk(&p.tmK, K, d, n, d, 64, 128, SW128) ||
         !tmap_bf16(&p.tmV, V, d, n, d, 64, 128, SW128))
         return TSP_ERR_CUDA;
     p.O = static_cast<__nv_bfloat16*>(O);
@@ -1269,8 +1287,10 @@ tsp_status_t launch_attn_core(const void* Q, const void* K, const void* V, int64
     {
         std::lock_guard<std::mutex> lk(g_mu);
         if (!attr_set[dev]) {
-            if (cudaFuncSetAttribute(attn_core_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     smem) != cudaSuccess)
+            if (cudaFuncSetAttribute(attn_core_kernel<true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+                cudaFuncSetAttribute(attn_core_kernel<false>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
                 return TSP_ERR_CUDA;
             attr_set[dev] = true;
         }
@@ -1278,7 +1298,10 @@ tsp_status_t launch_attn_core(const void* Q, const void* K, const void* V, int64
     const int grid = std::min(p.items, sms);
     TraceRec rec;
     const bool traced = trace_begin(st, &rec, causal ? "attn_core_causal" : "attn_core");
-    attn_core_kernel<<<grid, AttnCore::kThreads, smem, st>>>(p);
+    if (qk_f16)
+        attn_core_kernel<true><<<grid, AttnCore::kThreads, smem, st>>>(p);
+    else
+        attn_core_kernel<false><<<grid, AttnCore::kThreads, smem, st>>>(p);
     const cudaError_t e = cudaGetLastError();
     if (traced) trace_end(st, &rec);
     return e == cudaSuccess ? TSP_OK : TSP_ERR_CUDA;
@@ -1327,6 +1350,8 @@ const char* tsp_status_string(tsp_status_t s) {
         case TSP_ERR_CUDA: return "CUDA error";
         case TSP_ERR_TIMEOUT: return "a device-side wait timed out";
         case TSP_ERR_WORKSPACE: return "workspace missing or too small";
+        case TSP_ERR_RANGE:
+            return "a value left the range of an fp16 intermediate (saturated at 65504)";
         case TSP_ERR_SCRATCH_LIMIT:
             return "problem needs more scratch than the no-allocation entry point's static array";
     }
@@ -1527,7 +1552,7 @@ tsp_status_t tsp_attn_core(const void* Q, const void* K, const void* V, int64_t 
     int dev = 0;
     DevInfo di;
     TSP_TRY(current_device(&dev, &di));
-    return launch_attn_core(Q, K, V, n, d, n_heads, P, causal, O,
+    return launch_attn_core(Q, K, V, n, d, n_heads, P, causal, false, O,
                             reinterpret_cast<cudaStream_t>(stream), dev, di.sms);
 }
 
@@ -1567,14 +1592,16 @@ tsp_status_t tsp_attn_forward(const void* X, const void* Wq, const void* Wk, con
     // every parameter shard's columns of W_q, W_k, W_v, for every sequence
     // shard's tokens: the projections of all (shard, shard) pairs in one
     // launch each (no sum crosses shards)
-    TSP_TRY(gemm_bf16(X, Wq, n, d, d, Q, st, dev, di.sms, "attn_proj"));
-    TSP_TRY(gemm_bf16(X, Wk, n, d, d, K, st, dev, di.sms, "attn_proj"));
-    TSP_TRY(gemm_bf16(X, Wv, n, d, d, V, st, dev, di.sms, "attn_proj"));
+    // (Q and K in fp16: their rounding is the largest term of the block's
+    // error, and fp16 carries three more mantissa bits than bf16)
+    TSP_TRY(gemm_bf16(X, Wq, n, d, d, Q, true, st, dev, di.sms, "attn_proj"));
+    TSP_TRY(gemm_bf16(X, Wk, n, d, d, K, true, st, dev, di.sms, "attn_proj"));
+    TSP_TRY(gemm_bf16(X, Wv, n, d, d, V, false, st, dev, di.sms, "attn_proj"));
     // each sequence shard's queries over the key/value shards in ring order
-    TSP_TRY(launch_attn_core(Q, K, V, n, d, n_heads, P, causal, O, st, dev, di.sms));
+    TSP_TRY(launch_attn_core(Q, K, V, n, d, n_heads, P, causal, true, O, st, dev, di.sms));
     // Y_s = sum over parameter shards w (in order) of O_{s,w} . W_o[rows of w]:
     // the K loop runs over the head groups in order, summing in tensor memory
-    return gemm_bf16(O, Wo, n, d, d, Y, st, dev, di.sms, "attn_out_proj");
+    return gemm_bf16(O, Wo, n, d, d, Y, false, st, dev, di.sms, "attn_out_proj");
 }
 
 tsp_status_t tsp_trace_enable(int enable) {
@@ -1709,7 +1736,7 @@ tsp_status_t tsp_poll_device_error(tsp_stream_t stream) {
         const uint32_t zero = 0;
         if (cudaMemcpyToSymbol(tspmlp::g_device_error, &zero, sizeof(zero)) != cudaSuccess)
             return TSP_ERR_CUDA;
-        return TSP_ERR_TIMEOUT;
+        return (word & tspmlp::kDevErrTimeout) ? TSP_ERR_TIMEOUT : TSP_ERR_RANGE;
     }
     return TSP_OK;
 }
