@@ -418,7 +418,7 @@ __global__ void __launch_bounds__(AttnCore::kThreads, 1)
                     for (int e = 0; e < 32; ++e)
                         mx = fmaxf(mx, 32 * c + e < lim ? __uint_as_float(v[e]) : -INFINITY);
                 }
-                const float mb = mx * p.sl2;
+                const float mb = __fmul_rn(mx, p.sl2);
                 float alpha = 1.f;
                 bool resc = false;
                 if (mb > m_run + C::kRescaleLog2) {
@@ -463,8 +463,12 @@ __global__ void __launch_bounds__(AttnCore::kThreads, 1)
                     for (int e = 0; e < 32; e += 2) {
                         const float x0 = 32 * c + e < lim ? __uint_as_float(v[e]) : -INFINITY;
                         const float x1 = 32 * c + e + 1 < lim ? __uint_as_float(v[e + 1]) : -INFINITY;
-                        const float p0 = ex2_approx(fmaf(x0, p.sl2, -moff));
-                        const float p1 = ex2_approx(fmaf(x1, p.sl2, -moff));
+                        // the product rounded first, as m_run was: the row's maximum
+                        // then gives exactly 2^0 however large the scores are (a fused
+                        // multiply-add would subtract m_run's rounding error, which at
+                        // scores near 1e11 exceeds the exponent range)
+                        const float p0 = ex2_approx(__fmul_rn(x0, p.sl2) - moff);
+                        const float p1 = ex2_approx(__fmul_rn(x1, p.sl2) - moff);
                         ls += p0 + p1;
                         pk[e >> 1] = pack_bf16x2(p0, p1);
                     }

@@ -93,9 +93,9 @@ struct WgradPair {
         }
     }
     __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t rank, uint32_t acc,
-                                    int q, int lane) {
+                                    int q, int lane, uint32_t stg) {
         typename Base::Tile t1{2 * ti.mi + static_cast<int>(rank), ti.nj};
-        Base::epilogue(p, t1, acc, q, lane);
+        Base::epilogue(p, t1, acc, q, lane, stg);
     }
 };
 
@@ -161,10 +161,10 @@ struct DhPair {
         }
     }
     __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t rank, uint32_t acc,
-                                    int q, int lane) {
-        const int row = ti.mi * 256 + static_cast<int>(rank) * 128 + q * 32 + lane;
-        const bool row_ok = row < p.n;
-        const long long off = static_cast<long long>(row) * p.ld;
+                                    int q, int lane, uint32_t stg) {
+        const int wr0 = ti.mi * 256 + static_cast<int>(rank) * 128 + q * 32;  // warp's first row
+        const int nrows = min(32, p.n - wr0);
+        float* base = p.dH + static_cast<long long>(wr0) * p.ld;
         const uint32_t t0 = acc + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll 1
         for (int cc = 0; cc < 8; ++cc) {
@@ -172,7 +172,7 @@ struct DhPair {
             tmem_ld_32x32b_x32(t0 + 32 * cc, dh);
             tmem_ld_wait();
             const int c0 = ti.nj * 256 + 32 * cc;
-            if (row_ok && c0 < p.width) store_f32x32(p.dH + off + c0, dh, p.width - c0);
+            if (c0 < p.width) warp_store_f32x32(stg, base + c0, p.ld, nrows, dh, p.width - c0, lane);
         }
     }
 };
@@ -261,10 +261,13 @@ struct BwdGateUpPair {
         }
     }
     __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t rank, uint32_t acc,
-                                    int q, int lane) {
-        const int row = ti.mi * 256 + static_cast<int>(rank) * 128 + q * 32 + lane;
+                                    int q, int lane, uint32_t stg) {
+        const int wr0 = ti.mi * 256 + static_cast<int>(rank) * 128 + q * 32;  // warp's first row
+        const int row = wr0 + lane;
         const bool row_ok = row < p.n;
+        const int nrows = min(32, p.n - wr0);
         const long long off = static_cast<long long>(row) * p.ld;
+        const long long off0 = static_cast<long long>(wr0) * p.ld;
         const uint32_t t0 = acc + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll 1
         for (int cc = 0; cc < (ACT == 1 ? 4 : 8); ++cc) {
@@ -272,14 +275,19 @@ struct BwdGateUpPair {
             const int valid = p.width - c0;
             const bool live = row_ok && valid > 0;
             float dh[32];
-            if (live) load_dh(p.dH + off + c0, valid, dh);
+            if (live) {
+                load_dh(p.dH + off + c0, valid, dh);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) dh[i] = 0.0f;
+            }
             uint32_t g[32], ph[16], pg[16], pu[16];
             tmem_ld_32x32b_x32(t0 + 32 * cc, g);
             if (ACT == 1) {
                 uint32_t u[32];
                 tmem_ld_32x32b_x32(t0 + 128 + 32 * cc, u);
                 tmem_ld_wait();
-                if (!live) continue;
+                if (valid <= 0) continue;  // the same for the whole warp
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     float h[2], dgv[2], duv[2];
@@ -296,10 +304,10 @@ struct BwdGateUpPair {
                     pg[i] = pack_bf16x2(dgv[0], dgv[1]);
                     pu[i] = pack_bf16x2(duv[0], duv[1]);
                 }
-                store_bf16x32(p.dU + off + c0, pu, valid);
+                warp_store_16x32(stg, p.dU + off0 + c0, p.ld, nrows, pu, valid, lane);
             } else {
                 tmem_ld_wait();
-                if (!live) continue;
+                if (valid <= 0) continue;
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     float h[2], dgv[2];
@@ -314,8 +322,8 @@ struct BwdGateUpPair {
                     pg[i] = pack_bf16x2(dgv[0], dgv[1]);
                 }
             }
-            store_bf16x32(p.H + off + c0, ph, valid);
-            store_bf16x32(p.dG + off + c0, pg, valid);
+            warp_store_16x32(stg, p.H + off0 + c0, p.ld, nrows, ph, valid, lane);
+            warp_store_16x32(stg, p.dG + off0 + c0, p.ld, nrows, pg, valid, lane);
         }
     }
 };

@@ -174,12 +174,12 @@ struct DgradWgradPair {
         }
     }
     __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t rank, uint32_t acc,
-                                    int q, int lane) {
+                                    int q, int lane, uint32_t stg) {
         if (ti.kind == kDgrad) {
-            D::epilogue(p.d, ti.d, rank, acc, q, lane);
+            D::epilogue(p.d, ti.d, rank, acc, q, lane, stg);
         } else if (ti.kind == kWgrad) {
             typename W::Tile t1{2 * ti.wmi + static_cast<int>(rank), ti.wnj};
-            W::epilogue(p.w, t1, acc, q, lane);
+            W::epilogue(p.w, t1, acc, q, lane, stg);
         }
     }
 };

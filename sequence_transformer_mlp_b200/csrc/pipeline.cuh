@@ -41,11 +41,16 @@ namespace tspmlp {
 
 constexpr int kPipelineThreads = 192;
 
-// Bytes of dynamic shared memory a recipe needs (stages + barriers + slack
-// for 1024-byte alignment of the stage ring).
+// Each epilogue warp stages its 32 x 32 blocks for coalesced stores in 4 KB
+// of shared memory after the barriers (recipes.cuh: warp_store_*).
+constexpr int kEpiStageBytesPerWarp = 4096;
+constexpr int kEpiStageBytes = 4 * kEpiStageBytesPerWarp;
+
+// Bytes of dynamic shared memory a recipe needs (stages + barriers + the
+// epilogue staging buffers + slack for 1024-byte alignment of the stage ring).
 template <class R>
 constexpr int pipeline_smem_bytes() {
-    return R::kStages * R::kStageBytes + 256 + 1024;
+    return R::kStages * R::kStageBytes + 256 + kEpiStageBytes + 1024;
 }
 
 // Bounded wait that ignores the abort flag (used while draining).
@@ -186,6 +191,7 @@ __global__ void __launch_bounds__(kPipelineThreads, 1)
     } else {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;
+        const uint32_t stg = ring + S * R::kStageBytes + 256 + q * kEpiStageBytesPerWarp;
         int local = 0;
         for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++local) {
             const int buf = local % NB;
@@ -196,7 +202,7 @@ __global__ void __launch_bounds__(kPipelineThreads, 1)
             if (!ok) break;
             tc_fence_after();
             const auto ti = R::tile(p, t);
-            R::epilogue(p, ti, tmem_base + static_cast<uint32_t>(buf * R::kAccCols), q, lane);
+            R::epilogue(p, ti, tmem_base + static_cast<uint32_t>(buf * R::kAccCols), q, lane, stg);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty_bar(buf));

@@ -25,7 +25,8 @@
 //   void load(const Params&, const Tile&, int kb, uint32_t rank, uint32_t stage,
 //             uint32_t leader_full_bar)               (1 thread in each CTA)
 //   void mma(const Tile&, int kb, uint32_t stage, uint32_t acc)   (leader, 1 thread)
-//   void epilogue(const Params&, const Tile&, uint32_t rank, uint32_t acc, int q, int lane)
+//   void epilogue(const Params&, const Tile&, uint32_t rank, uint32_t acc, int q, int lane,
+//                 uint32_t stg)   (stg: the warp's 4 KB staging buffer for warp_store_*)
 #pragma once
 
 #include "pipeline.cuh"
@@ -35,7 +36,7 @@ namespace tspmlp {
 
 template <class R>
 constexpr int pair_smem_bytes() {
-    return R::kStages * R::kStageBytes + 256 + 1024;
+    return R::kStages * R::kStageBytes + 256 + kEpiStageBytes + 1024;
 }
 
 template <class R>
@@ -159,6 +160,7 @@ __global__ void __launch_bounds__(kPipelineThreads, 1)
     } else {
         // ------------------------------------------------------------ epilogue (both CTAs)
         const int q = warp & 3;
+        const uint32_t stg = ring + S * R::kStageBytes + 256 + q * kEpiStageBytesPerWarp;
         int local = 0;
         for (int t = pair; t < num_tiles; t += npairs, ++local) {
             const int buf = local % NB;
@@ -169,7 +171,7 @@ __global__ void __launch_bounds__(kPipelineThreads, 1)
             if (!ok) break;
             tc_fence_after();
             const auto ti = R::tile(p, t);
-            R::epilogue(p, ti, rank, tmem_base + static_cast<uint32_t>(buf) * kAccCols, q, lane);
+            R::epilogue(p, ti, rank, tmem_base + static_cast<uint32_t>(buf) * kAccCols, q, lane, stg);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
@@ -258,10 +260,10 @@ struct FwdHiddenPair {
         }
     }
     __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t rank, uint32_t acc,
-                                    int q, int lane) {
+                                    int q, int lane, uint32_t stg) {
         // the same per-row work as the single-CTA tile, on this CTA's 128 rows
         typename FwdHidden<ACT>::Tile t1{ti.s, 2 * ti.mi + static_cast<int>(rank), ti.nj};
-        FwdHidden<ACT>::epilogue(p, t1, acc, q, lane);
+        FwdHidden<ACT>::epilogue(p, t1, acc, q, lane, stg);
     }
 };
 
@@ -290,28 +292,47 @@ struct DownAccumPair {
                     // ring start (seg_begin + s) fs with rot_P)
         int kwrap;  // rot_P fs: the K loop's hidden units wrap at this column
         int arow;   // first A row of the pair's 256 rows
+        int half;   // -1 whole tile; 0 / 1: first / second half of a split tile's K loop
+        int kb0;    // first k-block of this unit
+        int nkb;    // k-blocks of this unit
+        int slot;   // split tiles: index of the tile among them
     };
     __host__ __device__ static int pair_mtiles(const SegGeom& g) { return (g.seg_rows + 255) >> 8; }
     __host__ __device__ static int ntiles_n(const Params& p) { return (p.n_out + BN - 1) / BN; }
-    __host__ __device__ static int num_tiles(const Params& p) {
+    __host__ __device__ static int whole_tiles(const Params& p) {
         return p.g.num_segs * pair_mtiles(p.g) * ntiles_n(p);
     }
-    __device__ static Tile tile(const Params& p, int t) {
+    __host__ __device__ static int kblocks(const Params& p) { return NSEG * ((p.kdim + kBK - 1) / kBK); }
+    // work units: the whole tiles before split_from, then two halves of each
+    // later tile (units split_from + 2 j and + 2 j + 1)
+    __host__ __device__ static int num_tiles(const Params& p) {
+        const int w = whole_tiles(p);
+        return p.split_from > 0 ? p.split_from + 2 * (w - p.split_from) : w;
+    }
+    __device__ static Tile tile(const Params& p, int u) {
+        int t = u, half = -1;
+        if (p.split_from > 0 && u >= p.split_from) {
+            const int j = u - p.split_from;
+            t = p.split_from + (j >> 1);
+            half = j & 1;
+        }
         const int mt = pair_mtiles(p.g), per_seg = mt * ntiles_n(p);
         const int s = t / per_seg, r = t - s * per_seg;
         const int nj = r / mt;
         const int mi = r - nj * mt;
+        const int nkb = kblocks(p), h0 = nkb >> 1;
         // everything the per-k-block loads need, computed once a tile
         return Tile{s, mi, nj,
                     p.rot_P > 0 ? (p.g.seg_begin + s) * p.g.fs : p.g.shard_col(s),
-                    p.rot_P * p.g.fs, s * p.g.seg_rows + mi * 256};
+                    p.rot_P * p.g.fs, s * p.g.seg_rows + mi * 256, half,
+                    half == 1 ? h0 : 0, half < 0 ? nkb : (half == 0 ? h0 : nkb - h0),
+                    t - p.split_from};
     }
-    __device__ static int num_kb(const Params& p, const Tile&) {
-        return NSEG * ((p.kdim + kBK - 1) / kBK);
-    }
+    __device__ static int num_kb(const Params&, const Tile& ti) { return ti.nkb; }
     __device__ static void prefetch(const Params& p) { Base::prefetch(p); }
     __device__ static void load(const Params& p, const Tile& ti, int kb, uint32_t rank, uint32_t st,
                                 uint32_t bar) {
+        kb += ti.kb0;  // the unit's k-blocks within the tile's K loop
         // K segment of this k-block (NSEG <= 2), without a division: this runs
         // once per k-block in the producer thread
         static_assert(NSEG == 1 || NSEG == 2, "one or two K segments");
@@ -361,9 +382,55 @@ struct DownAccumPair {
         }
     }
     __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t rank, uint32_t acc,
-                                    int q, int lane) {
-        Base::template store_rows<BN / 32>(p, ti.s, ti.mi * 256 + static_cast<int>(rank) * 128 + q * 32 + lane,
-                                           ti.nj * BN, acc + (static_cast<uint32_t>(q * 32) << 16));
+                                    int q, int lane, uint32_t stg) {
+        const int wr0 = ti.mi * 256 + static_cast<int>(rank) * 128 + q * 32;  // warp's first row
+        const uint32_t t0 = acc + (static_cast<uint32_t>(q * 32) << 16);
+        if (ti.half < 0) {
+            Base::template store_rows<BN / 32>(p, ti.s, wr0, lane, ti.nj * BN, t0, stg);
+            return;
+        }
+        // a split tile: this warp's 32 rows x 256 columns of the partial sum
+        float* part = p.part + static_cast<long long>(ti.slot) * (256 * 256) +
+                      (static_cast<int>(rank) * 128 + q * 32) * 256;
+        int* flag = p.flags + ti.slot * 8 + static_cast<int>(rank) * 4 + q;
+        if (ti.half == 0) {
+#pragma unroll 1
+            for (int cc = 0; cc < BN / 32; ++cc) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(t0 + 32 * cc, v);
+                tmem_ld_wait();
+                warp_store_f32x32(stg, part + 32 * cc, 256, 32, v, 32, lane);
+            }
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) st_release_gpu(flag, 1);
+            return;
+        }
+        // second half: wait (bounded) for the first half's rows of this warp,
+        // then round first-half + second-half sums to bf16
+        if (lane == 0) wait_flag_gpu(flag);
+        __syncwarp();
+        const int nrows = min(32, p.g.seg_rows - wr0);
+        const long long row0 = static_cast<long long>(p.g.seg_begin + ti.s) * p.g.seg_rows + wr0;
+        const float* prow = part + lane * 256;
+#pragma unroll 1
+        for (int cc = 0; cc < BN / 32; ++cc) {
+            uint32_t v[32], pk[16];
+            tmem_ld_32x32b_x32(t0 + 32 * cc, v);
+            tmem_ld_wait();
+            const int c0 = ti.nj * BN + 32 * cc;
+            const int valid = p.n_out - c0;
+            if (valid <= 0) continue;
+            const float4* a4 = reinterpret_cast<const float4*>(prow + 32 * cc);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float4 a = __ldcg(a4 + i);
+                pk[2 * i] = pack_bf16x2(a.x + __uint_as_float(v[4 * i]), a.y + __uint_as_float(v[4 * i + 1]));
+                pk[2 * i + 1] =
+                    pack_bf16x2(a.z + __uint_as_float(v[4 * i + 2]), a.w + __uint_as_float(v[4 * i + 3]));
+            }
+            warp_store_16x32(stg, p.out + row0 * p.ldo + c0, p.ldo, nrows, pk, valid, lane);
+        }
     }
 };
 

@@ -83,6 +83,119 @@ __device__ __forceinline__ void store_f32x32(float* dst, const uint32_t (&v)[32]
     }
 }
 
+// ----------------------------------------------------------------------------
+// warp-staged stores (coalesced): in the epilogues a thread owns one tile row,
+// so a plain vector store of a warp writes 16 bytes into each of 32 rows.
+// These helpers pass a warp's 32 rows x 32 columns through a per-warp buffer
+// in shared memory (4 KB) and write it out row after row: every store
+// instruction then covers whole 128-byte (fp32) or 64-byte (16-bit) row pieces
+// of 4 or 8 consecutive rows.  Warp-collective: every lane calls, with the
+// warp's common destination base, row pitch and valid column count; rows at
+// or past `nrows` are not written.
+
+__device__ __forceinline__ void sts_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                       uint32_t d) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+                 "r"(d)
+                 : "memory");
+}
+
+__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+
+// Flags between CTAs of one persistent grid (all resident): a release store,
+// and a bounded acquire wait for the value 1 (about two seconds of
+// %globaltimer; on expiry the device error word records a timeout and the
+// caller goes on).
+__device__ __forceinline__ void st_release_gpu(int* p, int v) {
+    asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void wait_flag_gpu(const int* p) {
+    auto ld = [p]() {
+        int v;
+        asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+        return v;
+    };
+    if (ld() == 1) return;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t i = 1;; ++i) {
+        asm volatile("nanosleep.u32 %0;" ::"r"(64u));
+        if (ld() == 1) return;
+        if ((i & 15u) == 0u && global_timer_ns() - t0 > kWaitLimitNs) {
+            atomicOr(&g_device_error, kDevErrTimeout);
+            return;
+        }
+    }
+}
+
+// Lane t holds v[0..32) for row t: base + t * ld + [0, valid).  Staged with
+// row t at stg + 128 t and its 16-byte chunk i at chunk i ^ (t % 8) (no bank
+// conflicts either way); written 4 rows an instruction, 8 lanes a row.
+__device__ __forceinline__ void warp_store_f32x32(uint32_t stg, float* base, long long ld, int nrows,
+                                                  const uint32_t (&v)[32], int valid, int lane) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        sts_v4(stg + lane * 128 + ((static_cast<uint32_t>(i) ^ (lane & 7)) << 4), v[4 * i],
+               v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    __syncwarp();
+    const int j = lane & 7, c = 4 * j;
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+        const int r = 4 * it + (lane >> 3);
+        const uint4 x = lds_v4(stg + r * 128 + ((static_cast<uint32_t>(j) ^ (r & 7)) << 4));
+        if (r < nrows) {
+            float* d = base + r * ld + c;
+            if (c + 4 <= valid) {
+                *reinterpret_cast<uint4*>(d) = x;
+            } else {
+                if (c < valid) d[0] = __uint_as_float(x.x);
+                if (c + 1 < valid) d[1] = __uint_as_float(x.y);
+                if (c + 2 < valid) d[2] = __uint_as_float(x.z);
+            }
+        }
+    }
+    __syncwarp();
+}
+
+// Lane t holds the packed pairs pk[0..16) (32 16-bit values) for row t:
+// base + t * ld + [0, valid).  Staged with row t at stg + 64 t and its 16-byte
+// chunk i at chunk i ^ ((t / 2) % 4); written 8 rows an instruction, 4 lanes a
+// row.  The values are moved as 16-bit words, whatever their format.
+__device__ __forceinline__ void warp_store_16x32(uint32_t stg, void* base, long long ld, int nrows,
+                                                 const uint32_t (&pk)[16], int valid, int lane) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        sts_v4(stg + lane * 64 + ((static_cast<uint32_t>(i) ^ ((lane >> 1) & 3)) << 4), pk[4 * i],
+               pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+    __syncwarp();
+    const int j = lane & 3, c = 8 * j;
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+        const int r = 8 * it + (lane >> 2);
+        const uint4 x = lds_v4(stg + r * 64 + ((static_cast<uint32_t>(j) ^ ((r >> 1) & 3)) << 4));
+        if (r < nrows) {
+            uint16_t* d = static_cast<uint16_t*>(base) + r * ld + c;
+            if (c + 8 <= valid) {
+                *reinterpret_cast<uint4*>(d) = x;
+            } else {
+                const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                for (int e = 0; e < 7; ++e)
+                    if (c + e < valid)
+                        d[e] = static_cast<uint16_t>((e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu));
+            }
+        }
+    }
+    __syncwarp();
+}
+
 // ============================================================================
 // K1: column-split gate/up projection with the activation fused.
 //   SwiGLU: H[:, j] = SiLU(X.W_gate[:, c+j]) * (X.W_up[:, c+j]), 128 columns a
@@ -156,10 +269,11 @@ struct FwdHidden {
             umma_bf16(acc, a, b, kIdesc, (kb | kk) != 0 ? 1u : 0u);
         }
     }
-    __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t acc, int q, int lane) {
-        const int rl = ti.mi * 128 + q * 32 + lane;
-        const bool row_ok = rl < p.g.seg_rows;
-        __nv_bfloat16* hrow = p.H + static_cast<long long>(ti.s * p.g.seg_rows + rl) * p.ldh;
+    __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t acc, int q, int lane,
+                                    uint32_t stg) {
+        const int wr0 = ti.mi * 128 + q * 32;  // the warp's first tile row
+        const int nrows = min(32, p.g.seg_rows - wr0);
+        __nv_bfloat16* hbase = p.H + static_cast<long long>(ti.s * p.g.seg_rows + wr0) * p.ldh;
         const uint32_t t0 = acc + (static_cast<uint32_t>(q * 32) << 16);
         if (ACT == 1) {
 #pragma unroll 1
@@ -176,7 +290,7 @@ struct FwdHidden {
                     pk[i] = pack_bf16x2(h0, h1);
                 }
                 const int c0 = ti.nj * 128 + 32 * cc;
-                if (row_ok) store_bf16x32(hrow + c0, pk, p.width - c0);
+                if (c0 < p.width) warp_store_16x32(stg, hbase + c0, p.ldh, nrows, pk, p.width - c0, lane);
             }
         } else {
 #pragma unroll 1
@@ -189,7 +303,7 @@ struct FwdHidden {
                     pk[i] = pack_bf16x2(gelu_f(__uint_as_float(z[2 * i])),
                                         gelu_f(__uint_as_float(z[2 * i + 1])));
                 const int c0 = ti.nj * 256 + 32 * cc;
-                if (row_ok) store_bf16x32(hrow + c0, pk, p.width - c0);
+                if (c0 < p.width) warp_store_16x32(stg, hbase + c0, p.ldh, nrows, pk, p.width - c0, lane);
             }
         }
     }
@@ -221,6 +335,14 @@ struct DownAccum {
         long long ldacc;
         __nv_bfloat16* out;  // [rows][n_out] bf16 (global rows)
         long long ldo;
+        // Tail split (paired kernel, mode 3 only): the tiles from split_from on
+        // -- fewer than half a wave -- each run as two halves of their K loop
+        // on two pairs; the first half leaves its fp32 sum in `part` and raises
+        // one flag per epilogue warp, the second adds it before rounding.
+        // split_from == 0: no split.
+        int split_from;
+        float* part;  // [split tiles][256][256] fp32
+        int* flags;   // [split tiles][8], zeroed before the launch
     };
     static constexpr const char* kName =
         B_MN ? "down_accum_fwd" : (NSEG == 2 ? "dgrad_accum_swiglu" : "dgrad_accum_gelu");
@@ -232,12 +354,19 @@ struct DownAccum {
             tma_prefetch_desc(&p.tmB1);
         }
     }
-    // One thread's accumulator row (tile row rl of segment s) over NCHUNK x 32
-    // columns starting at output column col0, applied in the launch's mode.
+    // A warp's 32 accumulator rows (tile rows wr0 .. wr0 + 31 of segment s,
+    // this thread's row wr0 + lane) over NCHUNK x 32 columns starting at output
+    // column col0, applied in the launch's mode.  The plain stores (modes 0, 3,
+    // 4) go through the warp's staging buffer; the read-modify-write modes
+    // (1, 2) keep one row a thread.
     template <int NCHUNK>
-    __device__ static void store_rows(const Params& p, int s, int rl, int col0, uint32_t t0) {
+    __device__ static void store_rows(const Params& p, int s, int wr0, int lane, int col0,
+                                      uint32_t t0, uint32_t stg) {
+        const int rl = wr0 + lane;
         const bool row_ok = rl < p.g.seg_rows;
-        const long long row = static_cast<long long>(p.g.seg_begin + s) * p.g.seg_rows + rl;
+        const int nrows = min(32, p.g.seg_rows - wr0);
+        const long long row0 = static_cast<long long>(p.g.seg_begin + s) * p.g.seg_rows + wr0;
+        const long long row = row0 + lane;
 #pragma unroll 1
         for (int cc = 0; cc < NCHUNK; ++cc) {
             uint32_t v[32];
@@ -245,10 +374,32 @@ struct DownAccum {
             tmem_ld_wait();
             const int c0 = col0 + 32 * cc;
             const int valid = p.n_out - c0;
-            if (!row_ok || valid <= 0) continue;
+            if (valid <= 0) continue;  // the same for the whole warp
             if (p.mode == 0) {
-                store_f32x32(p.acc + row * p.ldacc + c0, v, valid);
-            } else if (p.mode == 1) {
+                warp_store_f32x32(stg, p.acc + row0 * p.ldacc + c0, p.ldacc, nrows, v, valid, lane);
+                continue;
+            }
+            if (p.mode == 3 || p.mode == 4) {
+                uint32_t pk[16];
+                if (p.mode == 3) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+                } else {
+                    bool big = false;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float x0 = __uint_as_float(v[2 * i]), x1 = __uint_as_float(v[2 * i + 1]);
+                        big |= row_ok && (fabsf(x0) > 65504.f || fabsf(x1) > 65504.f);
+                        pk[i] = pack_f16x2_sat(x0, x1);
+                    }
+                    if (big) atomicOr(&g_device_error, kDevErrRange);
+                }
+                warp_store_16x32(stg, p.out + row0 * p.ldo + c0, p.ldo, nrows, pk, valid, lane);
+                continue;
+            }
+            if (!row_ok) continue;
+            if (p.mode == 1) {
                 float* a = p.acc + row * p.ldacc + c0;
                 if (valid >= 32) {
                     float4* a4 = reinterpret_cast<float4*>(a);
@@ -266,20 +417,9 @@ struct DownAccum {
                     for (int i = 0; i < 32; ++i)
                         if (i < valid) a[i] += __uint_as_float(v[i]);
                 }
-            } else if (p.mode == 4) {
+            } else {  // mode 2: bf16(acc + tile)
                 uint32_t pk[16];
-                bool big = false;
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float x0 = __uint_as_float(v[2 * i]), x1 = __uint_as_float(v[2 * i + 1]);
-                    big |= fabsf(x0) > 65504.f || fabsf(x1) > 65504.f;
-                    pk[i] = pack_f16x2_sat(x0, x1);
-                }
-                if (big) atomicOr(&g_device_error, kDevErrRange);
-                store_bf16x32(p.out + row * p.ldo + c0, pk, valid);  // 16-bit words, any format
-            } else {
-                uint32_t pk[16];
-                if (p.mode == 2) {
+                {
                     const float* a = p.acc + row * p.ldacc + c0;
                     if (valid >= 32) {
                         const float4* a4 = reinterpret_cast<const float4*>(a);
@@ -300,10 +440,6 @@ struct DownAccum {
                             pk[i] = pack_bf16x2(x0, x1);
                         }
                     }
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
                 }
                 store_bf16x32(p.out + row * p.ldo + c0, pk, valid);
             }
@@ -341,10 +477,11 @@ struct Wgrad {
         tma_prefetch_desc(&p.tmB0);
         if (SPLIT) tma_prefetch_desc(&p.tmB1);
     }
-    __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t acc, int q, int lane) {
-        const int rl = ti.mi * 128 + q * 32 + lane;
-        const bool row_ok = rl < p.m_valid;
-        const long long row = static_cast<long long>(p.out_row0 + rl);
+    __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t acc, int q, int lane,
+                                    uint32_t stg) {
+        const int wr0 = ti.mi * 128 + q * 32;  // the warp's first output row
+        const int nrows = min(32, p.m_valid - wr0);
+        const long long row0 = static_cast<long long>(p.out_row0 + wr0);
         const uint32_t t0 = acc + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll 1
         for (int cc = 0; cc < NCOLS / 32; ++cc) {
@@ -354,7 +491,9 @@ struct Wgrad {
             const int which = SPLIT ? cc / (NCOLS / 64) : 0;
             const int cl = ti.nj * kTileCols + 32 * (SPLIT ? cc % (NCOLS / 64) : cc);
             float* o = which ? p.out1 : p.out0;
-            if (row_ok) store_f32x32(o + row * p.ldo + p.out_col0 + cl, v, p.n_valid - cl);
+            if (cl < p.n_valid)
+                warp_store_f32x32(stg, o + row0 * p.ldo + p.out_col0 + cl, p.ldo, nrows, v,
+                                  p.n_valid - cl, lane);
         }
     }
 };

@@ -52,11 +52,13 @@ struct FwdHiddenSavePair : FwdHiddenPair<ACT> {
     }
 
     __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t rank, uint32_t acc,
-                                    int q, int lane) {
-        const int rl = (2 * ti.mi + static_cast<int>(rank)) * 128 + q * 32 + lane;
+                                    int q, int lane, uint32_t stg) {
+        const int wr0 = (2 * ti.mi + static_cast<int>(rank)) * 128 + q * 32;  // warp's first row
+        const int rl = wr0 + lane;
         const bool row_ok = rl < p.g.seg_rows;
+        const int nrows = min(32, p.g.seg_rows - wr0);
         const int r = ti.s * p.g.seg_rows + rl;
-        const long long off = static_cast<long long>(r) * p.ldh;
+        const long long off0 = static_cast<long long>(ti.s * p.g.seg_rows + wr0) * p.ldh;
         const uint32_t t0 = acc + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll 1
         for (int cc = 0; cc < Base::kOut / 32; ++cc) {
@@ -68,7 +70,7 @@ struct FwdHiddenSavePair : FwdHiddenPair<ACT> {
                 uint32_t u[32];
                 tmem_ld_32x32b_x32(t0 + 128 + 32 * cc, u);
                 tmem_ld_wait();
-                if (!row_ok || valid <= 0) continue;
+                if (valid <= 0) continue;  // the same for the whole warp
                 uint32_t pk[16], s1[32], s2[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
@@ -81,12 +83,14 @@ struct FwdHiddenSavePair : FwdHiddenPair<ACT> {
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
                     pk[i] = pack_bf16x2(__uint_as_float(g[2 * i]), __uint_as_float(g[2 * i + 1]));
-                store_bf16x32(p.H + off + c0, pk, valid);
-                store_factors(p.S1 + factor_index(r, c0, p.ldh), s1, valid);
-                store_factors(p.S2 + factor_index(r, c0, p.ldh), s2, valid);
+                warp_store_16x32(stg, p.H + off0 + c0, p.ldh, nrows, pk, valid, lane);
+                if (row_ok) {
+                    store_factors(p.S1 + factor_index(r, c0, p.ldh), s1, valid);
+                    store_factors(p.S2 + factor_index(r, c0, p.ldh), s2, valid);
+                }
             } else {
                 tmem_ld_wait();
-                if (!row_ok || valid <= 0) continue;
+                if (valid <= 0) continue;
                 uint32_t pk[16], s1[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
@@ -97,8 +101,8 @@ struct FwdHiddenSavePair : FwdHiddenPair<ACT> {
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
                     pk[i] = pack_bf16x2(__uint_as_float(g[2 * i]), __uint_as_float(g[2 * i + 1]));
-                store_bf16x32(p.H + off + c0, pk, valid);
-                store_factors(p.S1 + factor_index(r, c0, p.ldh), s1, valid);
+                warp_store_16x32(stg, p.H + off0 + c0, p.ldh, nrows, pk, valid, lane);
+                if (row_ok) store_factors(p.S1 + factor_index(r, c0, p.ldh), s1, valid);
             }
         }
     }
@@ -130,10 +134,12 @@ struct DhFactorPair : DhPair<ACT> {
     }
 
     __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t rank, uint32_t acc,
-                                    int q, int lane) {
-        const int row = ti.mi * 256 + static_cast<int>(rank) * 128 + q * 32 + lane;
+                                    int q, int lane, uint32_t stg) {
+        const int wr0 = ti.mi * 256 + static_cast<int>(rank) * 128 + q * 32;  // warp's first row
+        const int row = wr0 + lane;
         const bool row_ok = row < p.n;
-        const long long off = static_cast<long long>(row) * p.ld;
+        const int nrows = min(32, p.n - wr0);
+        const long long off0 = static_cast<long long>(wr0) * p.ld;
         const uint32_t t0 = acc + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll 1
         for (int cc = 0; cc < 8; ++cc) {
@@ -145,24 +151,27 @@ struct DhFactorPair : DhPair<ACT> {
                 const long long so = factor_index(row, c0, p.lds);
                 load_factors(p.S1 + so, valid, s1);
                 if (ACT == 1) load_factors(p.S2 + so, valid, s2);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) s1[i] = s2[i] = 0.0f;
             }
             uint32_t dh[32], pk[16];
             tmem_ld_32x32b_x32(t0 + 32 * cc, dh);
             tmem_ld_wait();
-            if (!live) continue;
+            if (valid <= 0) continue;  // the same for the whole warp
             if (ACT == 1) {
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
                     pk[i] = pack_bf16x2(__uint_as_float(dh[2 * i]) * s1[2 * i],
                                         __uint_as_float(dh[2 * i + 1]) * s1[2 * i + 1]);
-                store_bf16x32(p.dU + off + c0, pk, valid);
+                warp_store_16x32(stg, p.dU + off0 + c0, p.ld, nrows, pk, valid, lane);
             }
             const float(&sg)[32] = ACT == 1 ? s2 : s1;
 #pragma unroll
             for (int i = 0; i < 16; ++i)
                 pk[i] = pack_bf16x2(__uint_as_float(dh[2 * i]) * sg[2 * i],
                                     __uint_as_float(dh[2 * i + 1]) * sg[2 * i + 1]);
-            store_bf16x32(p.dG + off + c0, pk, valid);
+            warp_store_16x32(stg, p.dG + off0 + c0, p.ld, nrows, pk, valid, lane);
         }
     }
 };

@@ -184,44 +184,56 @@ void trace_end(cudaStream_t st, TraceRec* rec) {
 
 // Paired launch: clusters of two CTAs (cta_group::2 tiles), as many pairs as
 // can be resident at once, each walking the tile list persistently.
+// Pairs of recipe R that can be resident at once on device `dev` (sets the
+// kernel's shared-memory attribute on first use); 0 on a CUDA error.
+template <class R>
+int pair_capacity(int dev, int sms) {
+    constexpr int smem = pair_smem_bytes<R>();
+    static_assert(smem <= 232448, "stage ring exceeds 227 KB of shared memory");
+    static bool attr_set[kMaxDevices] = {};
+    static int max_pairs[kMaxDevices] = {};
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!attr_set[dev]) {
+        if (cudaFuncSetAttribute(umma_pair_pipeline_kernel<R>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return 0;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cudaLaunchConfig_t q = {};
+        q.gridDim = dim3(static_cast<unsigned>(sms / 2 * 2));
+        q.blockDim = dim3(kPipelineThreads);
+        q.dynamicSmemBytes = smem;
+        q.attrs = attr;
+        q.numAttrs = 1;
+        int nc = 0;
+        if (cudaOccupancyMaxActiveClusters(&nc, umma_pair_pipeline_kernel<R>, &q) != cudaSuccess ||
+            nc <= 0) {
+            cudaGetLastError();
+            nc = sms / 2;
+        }
+        max_pairs[dev] = nc;
+        attr_set[dev] = true;
+    }
+    return max_pairs[dev];
+}
+
 template <class R>
 tsp_status_t launch_pair(const typename R::Params& p, cudaStream_t st, int dev, int sms,
                          const char* trace_name = nullptr) {
     const int tiles = R::num_tiles(p);
     if (tiles <= 0) return TSP_OK;
     constexpr int smem = pair_smem_bytes<R>();
-    static_assert(smem <= 232448, "stage ring exceeds 227 KB of shared memory");
-    static bool attr_set[kMaxDevices] = {};
-    static int max_pairs[kMaxDevices] = {};
+    const int cap = pair_capacity<R>(dev, sms);
+    if (cap <= 0) return TSP_ERR_CUDA;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    {
-        std::lock_guard<std::mutex> lk(g_mu);
-        if (!attr_set[dev]) {
-            if (cudaFuncSetAttribute(umma_pair_pipeline_kernel<R>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     smem) != cudaSuccess)
-                return TSP_ERR_CUDA;
-            cudaLaunchConfig_t q = {};
-            q.gridDim = dim3(static_cast<unsigned>(sms / 2 * 2));
-            q.blockDim = dim3(kPipelineThreads);
-            q.dynamicSmemBytes = smem;
-            q.attrs = attr;
-            q.numAttrs = 1;
-            int nc = 0;
-            if (cudaOccupancyMaxActiveClusters(&nc, umma_pair_pipeline_kernel<R>, &q) != cudaSuccess ||
-                nc <= 0) {
-                cudaGetLastError();
-                nc = sms / 2;
-            }
-            max_pairs[dev] = nc;
-            attr_set[dev] = true;
-        }
-    }
-    const int pairs = std::min(tiles, max_pairs[dev]);
+    const int pairs = std::min(tiles, cap);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
     cfg.blockDim = dim3(kPipelineThreads);
@@ -399,12 +411,24 @@ struct FwdPlan {
     int tsp_group = 1;          // ring passes: sequence shards per launch
     int64_t row_group = 0;      // > 0: one-chunk passes over groups of this many token rows
     size_t h_bytes = 0, acc_bytes = 0;
+    // one-chunk passes: room for the down projection's tail split (the fp32
+    // partial sums and flags of up to kMaxSplitTiles tiles); 0 = no split
+    size_t split_bytes = 0;
     size_t total() const {
         if (fused) return align256(ring_bytes) + align256(sync_bytes);
         if (fused_passes) return 2 * align256(h_bytes) + align256(acc_bytes) + align256(sync_bytes);
-        return align256(h_bytes) + align256(acc_bytes);
+        return align256(h_bytes) + align256(acc_bytes) + split_bytes;
     }
 };
+
+// The down projection's tail split: when a launch's last wave of 256 x 256
+// tiles fills at most half the pairs, each of those tiles runs as two halves
+// of its K loop on two pairs (DownAccum::Params::split_from).  The area holds
+// the first halves' fp32 sums and one flag per epilogue warp.
+constexpr int kMaxSplitTiles = 64;
+constexpr size_t kSplitPartBytes = static_cast<size_t>(kMaxSplitTiles) * 256 * 256 * 4;
+constexpr size_t kSplitFlagBytes = static_cast<size_t>(kMaxSplitTiles) * 8 * 4;
+constexpr size_t kSplitBytes = kSplitPartBytes + 256 + kSplitFlagBytes + 256;
 
 // The fused schedule: row blocks of 128 tokens per sequence segment, grouped
 // GM at a time; the H ring holds three groups (R = 3*GM row-block slots, or one
@@ -521,9 +545,14 @@ FwdPlan plan_forward_budget(int64_t n, int64_t d, int64_t f, int P, tsp_dtype_t 
 FwdPlan plan_forward(int64_t n, int64_t d, int64_t f, int P, tsp_dtype_t dt, tsp_sched_t sched) {
     FwdPlan pl = plan_forward_budget(n, d, f, P, dt, sched, kFusedRingBudget);
     if (pl.fused) return pl;
-    return plan_forward_budget(n, d, f, P, dt, sched,
-                               sched == TSP_SCHED_SHARD_PASSES_FUSED ? kFusedPassesBudget
-                                                                     : kFwdHiddenBudget);
+    pl = plan_forward_budget(n, d, f, P, dt, sched,
+                             sched == TSP_SCHED_SHARD_PASSES_FUSED ? kFusedPassesBudget
+                                                                   : kFwdHiddenBudget);
+    // one-chunk weight-shard passes write Y directly: room for the tail split
+    if (dt == TSP_DT_BF16 && !pl.fused_passes && !pl.ring && pl.acc_bytes == 0 &&
+        (pl.row_group > 0 || pl.chunks.size() == 1))
+        pl.split_bytes = kSplitBytes;
+    return pl;
 }
 
 // The schedule for a caller workspace of ws_bytes: the preferred one if it
@@ -533,6 +562,11 @@ FwdPlan plan_forward_for(int64_t n, int64_t d, int64_t f, int P, tsp_dtype_t dt,
                          size_t ws_bytes) {
     FwdPlan pl = plan_forward(n, d, f, P, dt, sched);
     if (pl.total() <= ws_bytes || dt != TSP_DT_BF16) return pl;
+    if (pl.split_bytes > 0 && pl.total() - pl.split_bytes <= ws_bytes) {
+        pl.split_bytes = 0;  // the same passes without the tail split
+        return pl;
+    }
+    pl.split_bytes = 0;
     if (pl.fused) {
         const size_t sync = align256(pl.sync_bytes);
         if (ws_bytes <= sync + 256) {
@@ -604,7 +638,7 @@ tsp_status_t fwd_pass_bf16(const void* X, const void* Wg, const void* Wu, const 
                            int64_t n, int64_t d, int64_t f, const SegGeom& g, int64_t width,
                            int mode, __nv_bfloat16* H, float* acc, void* Y, cudaStream_t st,
                            int dev, int sms, int rot_P = 0, float* S1 = nullptr,
-                           float* S2 = nullptr) {
+                           float* S2 = nullptr, char* split_area = nullptr) {
     using K1 = FwdHidden<ACT>;
     using K2 = DownAccum<true, 1>;
     typename K1::Params p1;
@@ -645,7 +679,22 @@ tsp_status_t fwd_pass_bf16(const void* X, const void* Wg, const void* Wu, const 
     p2.ldacc = d;
     p2.out = static_cast<__nv_bfloat16*>(Y);
     p2.ldo = d;
-    return launch_pair<DownAccumPair<true, 1, 256>>(p2, st, dev, sms);
+    using D2 = DownAccumPair<true, 1, 256>;
+    if (split_area && mode == 3 && rot_P == 0) {
+        // a last wave of r tiles on at most half the pairs: each of its tiles
+        // as two halves of the K loop, so the wave takes half as long
+        const int T = D2::whole_tiles(p2), cap = pair_capacity<D2>(dev, sms);
+        const int r = cap > 0 ? T % cap : 0;
+        if (T > cap && r > 0 && 2 * r <= cap && r <= kMaxSplitTiles && D2::kblocks(p2) >= 2) {
+            p2.split_from = T - r;
+            p2.part = reinterpret_cast<float*>(split_area);
+            p2.flags = reinterpret_cast<int*>(split_area + kSplitPartBytes + 256);
+            if (cudaMemsetAsync(p2.flags, 0, static_cast<size_t>(r) * 8 * sizeof(int), st) !=
+                cudaSuccess)
+                return TSP_ERR_CUDA;
+        }
+    }
+    return launch_pair<D2>(p2, st, dev, sms);
 }
 
 // The whole forward as one persistent launch (fused.cuh).
@@ -806,6 +855,9 @@ tsp_status_t forward_bf16(const void* X, const void* Wg, const void* Wu, const v
     float* acc = pl.acc_bytes ? reinterpret_cast<float*>(static_cast<char*>(ws) +
                                                          align256(pl.h_bytes))
                               : nullptr;
+    char* split = pl.split_bytes ? static_cast<char*>(ws) + align256(pl.h_bytes) +
+                                       align256(pl.acc_bytes)
+                                 : nullptr;
     const int64_t fs = f / P;
     if (pl.row_group > 0) {
         // independent row groups: each a complete one-chunk pass on offset views
@@ -816,7 +868,7 @@ tsp_status_t forward_bf16(const void* X, const void* Wg, const void* Wu, const v
             void* Yg = static_cast<char*>(Y) + r0 * xe;
             const SegGeom g = seg_all_rows(rows, P, fs, 0);
             TSP_TRY(fwd_pass_bf16<ACT>(Xg, Wg, Wu, Wd, rows, d, f, g, f, 3, H, nullptr, Yg, st, dev,
-                                       sms));
+                                       sms, 0, nullptr, nullptr, split));
         }
         return TSP_OK;
     }
@@ -825,7 +877,8 @@ tsp_status_t forward_bf16(const void* X, const void* Wg, const void* Wu, const v
         for (int i = 0; i < np; ++i) {
             const SegGeom g = seg_all_rows(n, P, fs, pl.chunks[i].col_base);
             TSP_TRY(fwd_pass_bf16<ACT>(X, Wg, Wu, Wd, n, d, f, g, pl.chunks[i].width,
-                                       accum_mode(i, np), H, acc, Y, st, dev, sms));
+                                       accum_mode(i, np), H, acc, Y, st, dev, sms, 0, nullptr,
+                                       nullptr, split));
         }
     } else if (pl.ring_rotated) {
         for (int s0 = 0; s0 < P; s0 += pl.tsp_group) {

@@ -354,3 +354,24 @@ def test_llama70b_shape_sampled_rows():
     rows = cover_rows(LLAMA70B.n, 256, LLAMA70B.seed, groups=groups)
     assert {4096, 6143} <= set(rows) and len(rows) >= 32
     _sampled_check(LLAMA70B, inp, Y, rows)
+
+
+@pytest.mark.parametrize("act", ["swiglu", "gelu"])
+def test_bf16_down_projection_tail_split(act):
+    """80 down-projection tiles of 256 x 256 on 74 CTA pairs: the last wave's
+    6 tiles each run as two halves of their K loop on two pairs, the second
+    half adding the first's fp32 sum (the tail split).  Compared in full, and
+    with the same forward run without the split (a workspace without its
+    room), which differs only in the rounding of the split tiles."""
+    n, d, f, P = 10 * 256, 8 * 256, 8 * 128, 8
+    wl = small(act, "bf16", n, d, f, P, seed=81, w_std=0.03)
+    inp = make_inputs(wl)
+    Y = gpu_forward(inp, P, act)
+    ref = oracle.mlp_forward(inp["X"], inp["A"], inp["Wu"], inp["B"], act)
+    check(Y, ref, "bf16", "tail split")
+    Y2 = gpu_forward(inp, P, act, ws_bytes=n * f * 2)
+    check(Y2, ref, "bf16", "no tail split")
+    # tiles run column block by column block: the split ones are the last 6
+    # (rows 1024-2559 of columns 1792-2047); every other tile is bit-identical
+    assert np.array_equal(Y[:, :1792], Y2[:, :1792])
+    assert np.array_equal(Y[:1024], Y2[:1024])
