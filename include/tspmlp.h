@@ -262,7 +262,9 @@ TSP_API tsp_status_t tsp_mlp_workspace_size(int64_t n_tokens, int64_t d_model, i
  *
  * The saved buffer is opaque to the caller: H (row-major), then S1, then S2
  * (each over whole 32-row blocks, in the layout the two epilogues access
- * fastest), every region 256-byte aligned; tsp_mlp_saved_size gives its size.  It must be 256-byte
+ * fastest), then 16 MB of scratch the training forward's down projection uses
+ * as the forward's uses its workspace, every region 256-byte aligned;
+ * tsp_mlp_saved_size gives its size.  It must be 256-byte
  * aligned and overlap no other argument; the backward only reads it. */
 TSP_API tsp_status_t tsp_mlp_saved_size(int64_t n_tokens, int64_t d_model, int64_t d_ff, int P,
                                         tsp_act_t act, size_t* bytes);

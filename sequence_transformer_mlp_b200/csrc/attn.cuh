@@ -54,6 +54,13 @@ __device__ __forceinline__ void tmem_st_wait() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// The largest of three floats (one instruction on sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 // 2^x on the special-function unit (the ex2 instruction; -inf gives +0).
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;
@@ -407,16 +414,25 @@ __global__ void __launch_bounds__(AttnCore::kThreads, 1)
                     if (p.causal) lim = min(lim, qrow - kst + 1);
                 }
                 // pass 1: the row maximum of this block (32 columns at a time,
-                // so a thread holds one chunk of scores, not the whole row)
+                // so a thread holds one chunk of scores, not the whole row).  The
+                // loads are warp-collective; only the arithmetic branches on the
+                // mask, which only the last block of a shard and (causal) the
+                // diagonal blocks need.
+                const bool masked = lim < 128;
                 float mx = -INFINITY;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint32_t v[32];
                     tmem_ld_32x32b_x32(s_tm + 32 * c, v);
                     tmem_ld_wait();
+                    if (masked) {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        mx = fmaxf(mx, 32 * c + e < lim ? __uint_as_float(v[e]) : -INFINITY);
+                        for (int e = 0; e < 32; ++e)
+                            if (32 * c + e >= lim) v[e] = __float_as_uint(-INFINITY);
+                    }
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2)
+                        mx = fmax3(mx, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
                 }
                 const float mb = __fmul_rn(mx, p.sl2);
                 float alpha = 1.f;
@@ -452,25 +468,39 @@ __global__ void __launch_bounds__(AttnCore::kThreads, 1)
                 }
                 // pass 2: probabilities 2^(s log2(e)/sqrt(128) - m), their sum,
                 // and the P row as bf16 in the 128-byte-swizzled K-major layout
-                // (keys 64 b .. 64 b + 63 in box b; 16-byte chunk k at k ^ (r % 8))
+                // (keys 64 b .. 64 b + 63 in box b; 16-byte chunk k at k ^ (r % 8)).
+                // The exponent is one fused multiply-add: for the row's maximum it
+                // leaves only m's own rounding error, below 2^-12 while |m| <
+                // 4096.  Larger m (saturated inputs) take the product rounded
+                // first, as m was, so the maximum gives exactly 2^0.
+                const bool exact_max = fabsf(moff) >= 4096.f;
                 float ls = 0.f;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint32_t v[32], pk[16];
                     tmem_ld_32x32b_x32(s_tm + 32 * c, v);
                     tmem_ld_wait();
+                    if (masked) {
 #pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        const float x0 = 32 * c + e < lim ? __uint_as_float(v[e]) : -INFINITY;
-                        const float x1 = 32 * c + e + 1 < lim ? __uint_as_float(v[e + 1]) : -INFINITY;
-                        // the product rounded first, as m_run was: the row's maximum
-                        // then gives exactly 2^0 however large the scores are (a fused
-                        // multiply-add would subtract m_run's rounding error, which at
-                        // scores near 1e11 exceeds the exponent range)
-                        const float p0 = ex2_approx(__fmul_rn(x0, p.sl2) - moff);
-                        const float p1 = ex2_approx(__fmul_rn(x1, p.sl2) - moff);
-                        ls += p0 + p1;
-                        pk[e >> 1] = pack_bf16x2(p0, p1);
+                        for (int e = 0; e < 32; ++e)
+                            if (32 * c + e >= lim) v[e] = __float_as_uint(-INFINITY);
+                    }
+                    if (!exact_max) {
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) {
+                            const float p0 = ex2_approx(fmaf(__uint_as_float(v[e]), p.sl2, -moff));
+                            const float p1 = ex2_approx(fmaf(__uint_as_float(v[e + 1]), p.sl2, -moff));
+                            ls += p0 + p1;
+                            pk[e >> 1] = pack_bf16x2(p0, p1);
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) {
+                            const float p0 = ex2_approx(__fmul_rn(__uint_as_float(v[e]), p.sl2) - moff);
+                            const float p1 = ex2_approx(__fmul_rn(__uint_as_float(v[e + 1]), p.sl2) - moff);
+                            ls += p0 + p1;
+                            pk[e >> 1] = pack_bf16x2(p0, p1);
+                        }
                     }
                     const uint32_t box = p_row + (c >> 1) * 16384;
 #pragma unroll

@@ -919,7 +919,12 @@ tsp_status_t forward_bf16(const void* X, const void* Wg, const void* Wu, const v
 struct SavedLayout {
     size_t h = 0, s = 0;
     int nfac = 1;
-    size_t total() const { return h + nfac * s; }
+    // scratch for the down projection's tail split (as the forward's
+    // workspace has), so that the training forward's Y is the forward's bit
+    // for bit
+    size_t split = kSplitBytes;
+    size_t total() const { return h + nfac * s + split; }
+    size_t split_offset() const { return h + nfac * s; }
 };
 
 SavedLayout saved_layout(int64_t n, int64_t f, tsp_act_t act) {
@@ -961,7 +966,8 @@ tsp_status_t forward_train_bf16(const void* X, const void* Wg, const void* Wu, c
         // at the same offset r0 x f as its rows of H
         const int64_t ho = r0 * f;
         TSP_TRY(fwd_pass_bf16<ACT>(Xg, Wg, Wu, Wd, rows, d, f, g, f, /*mode direct*/ 3, H + ho,
-                                   nullptr, Yg, st, dev, sms, 0, S1 + ho, S2 ? S2 + ho : nullptr));
+                                   nullptr, Yg, st, dev, sms, 0, S1 + ho, S2 ? S2 + ho : nullptr,
+                                   base + sl.split_offset()));
     }
     return TSP_OK;
 }
