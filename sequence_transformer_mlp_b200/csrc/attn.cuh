@@ -101,7 +101,7 @@ struct AttnItem {
 };
 
 struct AttnCore {
-    static constexpr int kThreads = 320;
+    static constexpr int kThreads = 576;
     static constexpr int kTileBytes = 128 * 128 * 2;  // a 128 x 128 bf16 tile (two 64-column boxes)
     static constexpr int kStages = 3;
     static constexpr int kQOff = 0, kPOff = 2 * kTileBytes, kKVOff = 4 * kTileBytes;
@@ -198,8 +198,8 @@ __global__ void __launch_bounds__(AttnCore::kThreads, 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(s_full(a), 1);
-            mbar_init(s_empty(a), 4);
-            mbar_init(p_full(a), 4);
+            mbar_init(s_empty(a), 8);
+            mbar_init(p_full(a), 8);
             mbar_init(pv_done(a), 1);
         }
         mbar_init(drain_bar, 1);
@@ -377,15 +377,23 @@ __global__ void __launch_bounds__(AttnCore::kThreads, 1)
         }
         __syncwarp();
     } else {
-        // ---------------------------------------------------------------- softmax (two warpgroups)
-        const int a = (warp - 2) >> 2;            // tile of this warpgroup
+        // ---------------------------------------------------------------- softmax (four warpgroups)
+        // Two warpgroups per tile: both read the whole score row for its
+        // maximum (cheap), and each exponentiates, sums and writes P for one
+        // half of the 128 keys, and owns that half of O's columns.
+        const int sw = warp - 2;
+        const int a = sw >> 3;                    // tile of this warpgroup
+        const int hf = (sw >> 2) & 1;             // key half [64 hf, 64 hf + 64)
         const int q = warp & 3;                   // TMEM lane quarter
         const int r = q * 32 + lane;              // row of the tile
         const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
         const uint32_t s_tm = tmem + 256 + 128 * a + lane_off;
-        const uint32_t o_tm = tmem + 128 * a + lane_off;
-        const uint32_t p_row = ps + a * C::kTileBytes + r * 128;
+        const uint32_t o_tm = tmem + 128 * a + 64 * hf + lane_off;
+        const uint32_t p_box = ps + a * C::kTileBytes + hf * 16384;  // this half's P box
+        const uint32_t p_row = p_box + r * 128;
+        const uint32_t p_row_other = ps + a * C::kTileBytes + (1 - hf) * 16384 + r * 128;
         const uint32_t swz = static_cast<uint32_t>(r & 7);
+        const uint32_t bar_id = 1u + static_cast<uint32_t>(a * 4 + q);  // the row's two warps
         uint32_t s_cnt = 0, pv_cnt = 0;
         bool ok = true;
         for (int rd = 0; rd < rounds && ok; ++rd) {
@@ -413,27 +421,32 @@ __global__ void __launch_bounds__(AttnCore::kThreads, 1)
                     lim = kval;
                     if (p.causal) lim = min(lim, qrow - kst + 1);
                 }
-                // pass 1: the row maximum of this block (32 columns at a time,
-                // so a thread holds one chunk of scores, not the whole row).  The
-                // loads are warp-collective; only the arithmetic branches on the
-                // mask, which only the last block of a shard and (causal) the
-                // diagonal blocks need.
                 const bool masked = lim < 128;
-                float mx = -INFINITY;
+                // pass 1: the row maximum over all 128 keys (both warpgroups of
+                // the tile compute it, identically), two 32-column chunks per
+                // TMEM wait and four running maxima
+                // (one 32-column chunk per TMEM wait here: this kernel's 18 warps
+                // leave 96 registers a thread)
+                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    uint32_t v[32];
-                    tmem_ld_32x32b_x32(s_tm + 32 * c, v);
+                    uint32_t va[32];
+                    tmem_ld_32x32b_x32(s_tm + 32 * c, va);
                     tmem_ld_wait();
                     if (masked) {
 #pragma unroll
                         for (int e = 0; e < 32; ++e)
-                            if (32 * c + e >= lim) v[e] = __float_as_uint(-INFINITY);
+                            if (32 * c + e >= lim) va[e] = __float_as_uint(-INFINITY);
                     }
 #pragma unroll
-                    for (int e = 0; e < 32; e += 2)
-                        mx = fmax3(mx, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+                    for (int e = 0; e < 32; e += 8) {
+                        m4[0] = fmax3(m4[0], __uint_as_float(va[e]), __uint_as_float(va[e + 1]));
+                        m4[1] = fmax3(m4[1], __uint_as_float(va[e + 2]), __uint_as_float(va[e + 3]));
+                        m4[2] = fmax3(m4[2], __uint_as_float(va[e + 4]), __uint_as_float(va[e + 5]));
+                        m4[3] = fmax3(m4[3], __uint_as_float(va[e + 6]), __uint_as_float(va[e + 7]));
+                    }
                 }
+                const float mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
                 const float mb = __fmul_rn(mx, p.sl2);
                 float alpha = 1.f;
                 bool resc = false;
@@ -455,7 +468,7 @@ __global__ void __launch_bounds__(AttnCore::kThreads, 1)
                     tc_fence_after();
                     if (__any_sync(0xffffffffu, resc)) {
 #pragma unroll 1
-                        for (int c = 0; c < 4; ++c) {
+                        for (int c = 0; c < 2; ++c) {
                             uint32_t o[32];
                             tmem_ld_32x32b_x32(o_tm + 32 * c, o);
                             tmem_ld_wait();
@@ -466,51 +479,54 @@ __global__ void __launch_bounds__(AttnCore::kThreads, 1)
                         tmem_st_wait();
                     }
                 }
-                // pass 2: probabilities 2^(s log2(e)/sqrt(128) - m), their sum,
-                // and the P row as bf16 in the 128-byte-swizzled K-major layout
-                // (keys 64 b .. 64 b + 63 in box b; 16-byte chunk k at k ^ (r % 8)).
+                // pass 2 (this half's 64 keys): probabilities 2^(s log2(e)/sqrt(128)
+                // - m), their sum, and P as bf16 in the 128-byte-swizzled K-major
+                // layout (box hf; 16-byte chunk k of row r at chunk k ^ (r % 8)).
                 // The exponent is one fused multiply-add: for the row's maximum it
                 // leaves only m's own rounding error, below 2^-12 while |m| <
                 // 4096.  Larger m (saturated inputs) take the product rounded
                 // first, as m was, so the maximum gives exactly 2^0.
                 const bool exact_max = fabsf(moff) >= 4096.f;
-                float ls = 0.f;
+                float ls4[4] = {0.f, 0.f, 0.f, 0.f};
+                uint32_t v[2][32];
+                tmem_ld_32x32b_x32(s_tm + 64 * hf, v[0]);
+                tmem_ld_32x32b_x32(s_tm + 64 * hf + 32, v[1]);
+                tmem_ld_wait();
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t v[32], pk[16];
-                    tmem_ld_32x32b_x32(s_tm + 32 * c, v);
-                    tmem_ld_wait();
+                for (int c = 0; c < 2; ++c) {
+                    const int col0 = 64 * hf + 32 * c;
+                    uint32_t(&w)[32] = v[c];
+                    uint32_t pk[16];
                     if (masked) {
 #pragma unroll
                         for (int e = 0; e < 32; ++e)
-                            if (32 * c + e >= lim) v[e] = __float_as_uint(-INFINITY);
+                            if (col0 + e >= lim) w[e] = __float_as_uint(-INFINITY);
                     }
                     if (!exact_max) {
 #pragma unroll
                         for (int e = 0; e < 32; e += 2) {
-                            const float p0 = ex2_approx(fmaf(__uint_as_float(v[e]), p.sl2, -moff));
-                            const float p1 = ex2_approx(fmaf(__uint_as_float(v[e + 1]), p.sl2, -moff));
-                            ls += p0 + p1;
+                            const float p0 = ex2_approx(fmaf(__uint_as_float(w[e]), p.sl2, -moff));
+                            const float p1 = ex2_approx(fmaf(__uint_as_float(w[e + 1]), p.sl2, -moff));
+                            ls4[(e >> 1) & 3] += p0 + p1;
                             pk[e >> 1] = pack_bf16x2(p0, p1);
                         }
                     } else {
 #pragma unroll
                         for (int e = 0; e < 32; e += 2) {
-                            const float p0 = ex2_approx(__fmul_rn(__uint_as_float(v[e]), p.sl2) - moff);
-                            const float p1 = ex2_approx(__fmul_rn(__uint_as_float(v[e + 1]), p.sl2) - moff);
-                            ls += p0 + p1;
+                            const float p0 = ex2_approx(__fmul_rn(__uint_as_float(w[e]), p.sl2) - moff);
+                            const float p1 = ex2_approx(__fmul_rn(__uint_as_float(w[e + 1]), p.sl2) - moff);
+                            ls4[(e >> 1) & 3] += p0 + p1;
                             pk[e >> 1] = pack_bf16x2(p0, p1);
                         }
                     }
-                    const uint32_t box = p_row + (c >> 1) * 16384;
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const uint32_t chunk = static_cast<uint32_t>((c & 1) * 4 + k);
-                        st_shared_v4(box + ((chunk ^ swz) << 4), pk[4 * k], pk[4 * k + 1],
-                                     pk[4 * k + 2], pk[4 * k + 3]);
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint32_t chunk = static_cast<uint32_t>(c * 4 + kk);
+                        st_shared_v4(p_row + ((chunk ^ swz) << 4), pk[4 * kk], pk[4 * kk + 1],
+                                     pk[4 * kk + 2], pk[4 * kk + 3]);
                     }
                 }
-                lsum = lsum * alpha + ls;
+                lsum = lsum * alpha + ((ls4[0] + ls4[1]) + (ls4[2] + ls4[3]));
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(s_empty(a));
@@ -520,17 +536,26 @@ __global__ void __launch_bounds__(AttnCore::kThreads, 1)
                 if (lane == 0) mbar_arrive(p_full(a));
             }
             if (!ok) break;
-            // epilogue: O / l, bf16, this row of the item's head
+            // epilogue: the row sum of both halves, then this half's columns of
+            // O / l in bf16
             int w3 = 0;
             if (lane == 0) w3 = mbar_wait(pv_done(a), pv_cnt & 1u, abort_flag) ? 1 : 0;
             ++pv_cnt;
             if (!__shfl_sync(0xffffffffu, w3, 0)) break;
             tc_fence_after();
-            const float inv = 1.f / lsum;
+            // the last P V has read P: each half leaves its partial sum in its
+            // own P row, the row's two warps meet, read the other's, and meet
+            // again before either writes P of the next item there
+            asm volatile("st.shared.f32 [%0], %1;" ::"r"(p_row), "f"(lsum) : "memory");
+            asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
+            float lo;
+            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(lo) : "r"(p_row_other) : "memory");
+            asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
+            const float inv = 1.f / (hf == 0 ? lsum + lo : lo + lsum);
             const bool row_ok = qrow <= it.qlast;
-            __nv_bfloat16* orow = p.O + static_cast<long long>(qrow) * p.ldo + it.h * 128;
+            __nv_bfloat16* orow = p.O + static_cast<long long>(qrow) * p.ldo + it.h * 128 + 64 * hf;
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 2; ++c) {
                 uint32_t o[32];
                 tmem_ld_32x32b_x32(o_tm + 32 * c, o);
                 tmem_ld_wait();
