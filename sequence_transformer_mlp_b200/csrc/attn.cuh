@@ -336,27 +336,23 @@ __global__ void __launch_bounds__(AttnCore::kThreads, 1)
                 }
                 if (!ok) break;
                 umma_commit(kv_empty(kst));
+                // per block j and tile a: S_{a, j+1} as soon as the softmax has
+                // read S_{a, j} (it reads S first), then O_a += P_{a, j} V_j once
+                // the probabilities are in shared memory; the next block's
+                // scores are then ready when the softmax finishes this one
                 for (int j = 0; j < it.nkv && ok; ++j) {
                     if (!wait_kv(&vst)) {
                         ok = false;
                         break;
                     }
                     const bool more = j + 1 < it.nkv;
+                    if (more && !wait_kv(&kst)) {
+                        ok = false;
+                        break;
+                    }
 #pragma unroll
                     for (int a = 0; a < 2; ++a) {
-                        if (!mbar_wait(p_full(a), p_cnt[a] & 1u, abort_flag)) {
-                            ok = false;
-                            break;
-                        }
-                        ++p_cnt[a];
-                        tc_fence_after();
-                        issue_pv(a, vst, j > 0);
-                        if (a == 1) umma_commit(kv_empty(vst));
                         if (more) {
-                            if (a == 0 && !wait_kv(&kst)) {
-                                ok = false;
-                                break;
-                            }
                             if (!mbar_wait(s_empty(a), (s_cnt[a] & 1u) ^ 1u, abort_flag)) {
                                 ok = false;
                                 break;
@@ -366,6 +362,14 @@ __global__ void __launch_bounds__(AttnCore::kThreads, 1)
                             ++s_cnt[a];
                             if (a == 1) umma_commit(kv_empty(kst));
                         }
+                        if (!mbar_wait(p_full(a), p_cnt[a] & 1u, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        ++p_cnt[a];
+                        tc_fence_after();
+                        issue_pv(a, vst, j > 0);
+                        if (a == 1) umma_commit(kv_empty(vst));
                     }
                 }
                 if (!ok) break;
@@ -492,6 +496,11 @@ __global__ void __launch_bounds__(AttnCore::kThreads, 1)
                 tmem_ld_32x32b_x32(s_tm + 64 * hf, v[0]);
                 tmem_ld_32x32b_x32(s_tm + 64 * hf + 32, v[1]);
                 tmem_ld_wait();
+                // S_a is no longer read: the next block's Q K^T may overwrite it
+                // while these probabilities are computed
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(s_empty(a));
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
                     const int col0 = 64 * hf + 32 * c;
@@ -527,9 +536,6 @@ __global__ void __launch_bounds__(AttnCore::kThreads, 1)
                     }
                 }
                 lsum = lsum * alpha + ((ls4[0] + ls4[1]) + (ls4[2] + ls4[3]));
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(s_empty(a));
                 fence_proxy_async_smem();
                 tc_fence_before();
                 __syncwarp();
