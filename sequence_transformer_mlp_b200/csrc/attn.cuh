@@ -336,6 +336,9 @@ __global__ void __launch_bounds__(AttnCore::kThreads, 1)
                 }
                 if (!ok) break;
                 umma_commit(kv_empty(kst));
+                // Q is free once the item's last Q K^T is done: the next item's
+                // query tiles load while this item's last blocks finish
+                if (it.nkv == 1) umma_commit(q_empty);
                 // per block j and tile a: S_{a, j+1} as soon as the softmax has
                 // read S_{a, j} (it reads S first), then O_a += P_{a, j} V_j once
                 // the probabilities are in shared memory; the next block's
@@ -360,7 +363,10 @@ __global__ void __launch_bounds__(AttnCore::kThreads, 1)
                             tc_fence_after();
                             issue_s(a, kst);
                             ++s_cnt[a];
-                            if (a == 1) umma_commit(kv_empty(kst));
+                            if (a == 1) {
+                                umma_commit(kv_empty(kst));
+                                if (j + 2 == it.nkv) umma_commit(q_empty);
+                            }
                         }
                         if (!mbar_wait(p_full(a), p_cnt[a] & 1u, abort_flag)) {
                             ok = false;
@@ -373,7 +379,6 @@ __global__ void __launch_bounds__(AttnCore::kThreads, 1)
                     }
                 }
                 if (!ok) break;
-                umma_commit(q_empty);
                 ++done;
             }
             umma_commit(drain_bar);
