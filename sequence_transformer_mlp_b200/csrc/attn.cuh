@@ -247,26 +247,30 @@ __global__ void __launch_bounds__(AttnCore::kThreads, 1)
                 }
                 q_armed = true;
                 q_par = done & 1;
-                for (int t = 0; t < it.nkv && ok; ++t) {
+                // K_0, then K_{t+1} ahead of V_t: a key block's stage is the one
+                // the value block two blocks back used, so the keys of the next
+                // block load a whole block before the scores need them
+                auto load_block = [&](bool is_v, int t) {
                     int kst, kval;
                     C::block(p, it, t, &kst, &kval);
-                    for (int kv = 0; kv < 2; ++kv) {  // the key block, then the value block
-                        if (!mbar_wait(kv_empty(stage), phase ^ 1u, abort_flag)) {
-                            ok = false;
-                            break;
-                        }
-                        const CUtensorMap* m = kv ? &p.tmV : &p.tmK;
-                        const uint32_t dst = kvs + stage * C::kTileBytes;
-                        mbar_arrive_expect_tx(kv_full(stage), C::kTileBytes);
-                        tma_load_2d(dst, m, kv_full(stage), col, kst);
-                        tma_load_2d(dst + 16384, m, kv_full(stage), col + 64, kst);
-                        armed |= 1u << stage;
-                        armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
-                        if (++stage == S) {
-                            stage = 0;
-                            phase ^= 1u;
-                        }
+                    if (!mbar_wait(kv_empty(stage), phase ^ 1u, abort_flag)) return false;
+                    const CUtensorMap* m = is_v ? &p.tmV : &p.tmK;
+                    const uint32_t dst = kvs + stage * C::kTileBytes;
+                    mbar_arrive_expect_tx(kv_full(stage), C::kTileBytes);
+                    tma_load_2d(dst, m, kv_full(stage), col, kst);
+                    tma_load_2d(dst + 16384, m, kv_full(stage), col + 64, kst);
+                    armed |= 1u << stage;
+                    armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+                    if (++stage == S) {
+                        stage = 0;
+                        phase ^= 1u;
                     }
+                    return true;
+                };
+                ok = load_block(false, 0);
+                for (int t = 0; t < it.nkv && ok; ++t) {
+                    if (t + 1 < it.nkv && !load_block(false, t + 1)) ok = false;
+                    else if (!load_block(true, t)) ok = false;
                 }
                 ++done;
             }
@@ -344,12 +348,13 @@ __global__ void __launch_bounds__(AttnCore::kThreads, 1)
                 // the probabilities are in shared memory; the next block's
                 // scores are then ready when the softmax finishes this one
                 for (int j = 0; j < it.nkv && ok; ++j) {
-                    if (!wait_kv(&vst)) {
+                    // the producer's order: K_{j+1}, then V_j
+                    const bool more = j + 1 < it.nkv;
+                    if (more && !wait_kv(&kst)) {
                         ok = false;
                         break;
                     }
-                    const bool more = j + 1 < it.nkv;
-                    if (more && !wait_kv(&kst)) {
+                    if (!wait_kv(&vst)) {
                         ok = false;
                         break;
                     }
