@@ -348,13 +348,10 @@ __global__ void __launch_bounds__(AttnCore::kThreads, 1)
                 // the probabilities are in shared memory; the next block's
                 // scores are then ready when the softmax finishes this one
                 for (int j = 0; j < it.nkv && ok; ++j) {
-                    // the producer's order: K_{j+1}, then V_j
+                    // the producer's order: K_{j+1}, then V_j (waited for only
+                    // once the first tile's next scores are issued)
                     const bool more = j + 1 < it.nkv;
                     if (more && !wait_kv(&kst)) {
-                        ok = false;
-                        break;
-                    }
-                    if (!wait_kv(&vst)) {
                         ok = false;
                         break;
                     }
@@ -372,6 +369,10 @@ __global__ void __launch_bounds__(AttnCore::kThreads, 1)
                                 umma_commit(kv_empty(kst));
                                 if (j + 2 == it.nkv) umma_commit(q_empty);
                             }
+                        }
+                        if (a == 0 && !wait_kv(&vst)) {
+                            ok = false;
+                            break;
                         }
                         if (!mbar_wait(p_full(a), p_cnt[a] & 1u, abort_flag)) {
                             ok = false;
