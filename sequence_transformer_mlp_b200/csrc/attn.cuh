@@ -11,21 +11,26 @@
 // merge), so no shard ever needs the whole score row at once.  With the
 // causal mask the shards after s hold only future keys and are skipped.
 //
-// One CTA per SM, persistent, 320 threads:
+// One CTA per SM, persistent, 576 threads:
 //   warp 0      TMA producer: per work item the two 128-row query tiles, then
-//               the key and value blocks in the item's ring order through a
-//               ring of three 32 KB stages.
+//               the key and value blocks in the item's ring order (each key
+//               block one block ahead of its value block) through a ring of
+//               three 32 KB stages.
 //   warp 1      MMA issuer: S_a = Q_a K^T into tensor memory and O_a += P_a V
-//               (a = 0, 1), interleaved so that the tensor pipe works on one
-//               tile while the other tile's softmax runs.
-//   warps 2-5   softmax of tile 0, warps 6-9 softmax of tile 1: thread = one
-//               query row (warp w reads TMEM lanes 32 (w % 4) .. +31).  Reads
-//               its 128 scores, applies the mask, updates the running max
-//               (rescaling O in tensor memory only when the max grows by more
-//               than 2^8, which keeps every probability <= 256 and the result
-//               exact), writes the probabilities as bf16 to shared memory for
-//               the P V product, and at the end of the item divides O by the
-//               row sum and stores it.
+//               (a = 0, 1).  A tile's next scores are issued as soon as its
+//               softmax has read the current ones, so the tensor pipe works on
+//               one tile while the other tile's softmax runs.
+//   warps 2-17  softmax: two warpgroups per tile, one per half of the 128 keys
+//               of a block; thread = one query row (warp w reads TMEM lanes
+//               32 (w % 4) .. +31).  Each reads the row's 128 scores in two
+//               64-column rounds (the other half's for the maximum only, then
+//               its own, kept in registers), applies the mask, updates the
+//               running max (rescaling its half of O in tensor memory only
+//               when the max grows by more than 2^8, which keeps every
+//               probability <= 256 and the result exact), writes its half's
+//               probabilities as bf16 to shared memory for the P V product,
+//               and at the end of the item divides O by the row sum and stores
+//               it.
 // Tensor memory: O_0, O_1, S_0, S_1, 128 fp32 columns each (512 columns).
 // Shared memory: Q_0, Q_1, P_0, P_1 (32 KB each) and the K/V ring (96 KB).
 // Every wait is bounded as in pipeline.cuh.
@@ -59,6 +64,37 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float r;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
     return r;
+}
+
+// Two floats as one 64-bit register pair (the operand of the packed f32x2
+// instructions of sm_100).
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+// (d0, d1) = (a0, a1) * b + c, b and c packed pairs: one fma.rn.f32x2 (each
+// lane rounded once, as fmaf).
+__device__ __forceinline__ void fma_f32x2(float a0, float a1, uint64_t b, uint64_t c, float& d0,
+                                          float& d1) {
+    asm("{\n\t.reg .b64 va, vd;\n\t"
+        "mov.b64 va, {%2, %3};\n\t"
+        "fma.rn.f32x2 vd, va, %4, %5;\n\t"
+        "mov.b64 {%0, %1}, vd;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "l"(b), "l"(c));
+}
+
+// (s0, s1) += (b0, b1): one add.rn.f32x2.
+__device__ __forceinline__ void add_f32x2(float& s0, float& s1, float b0, float b1) {
+    asm("{\n\t.reg .b64 vs, vb;\n\t"
+        "mov.b64 vs, {%0, %1};\n\t"
+        "mov.b64 vb, {%2, %3};\n\t"
+        "add.rn.f32x2 vs, vs, vb;\n\t"
+        "mov.b64 {%0, %1}, vs;\n\t}"
+        : "+f"(s0), "+f"(s1)
+        : "f"(b0), "f"(b1));
 }
 
 // 2^x on the special-function unit (the ex2 instruction; -inf gives +0).
@@ -394,8 +430,8 @@ __global__ void __launch_bounds__(AttnCore::kThreads, 1)
     } else {
         // ---------------------------------------------------------------- softmax (four warpgroups)
         // Two warpgroups per tile: both read the whole score row for its
-        // maximum (cheap), and each exponentiates, sums and writes P for one
-        // half of the 128 keys, and owns that half of O's columns.
+        // maximum, and each exponentiates, sums and writes P for one half of
+        // the 128 keys, and owns that half of O's columns.
         const int sw = warp - 2;
         const int a = sw >> 3;                    // tile of this warpgroup
         const int hf = (sw >> 2) & 1;             // key half [64 hf, 64 hf + 64)
@@ -437,30 +473,40 @@ __global__ void __launch_bounds__(AttnCore::kThreads, 1)
                     if (p.causal) lim = min(lim, qrow - kst + 1);
                 }
                 const bool masked = lim < 128;
-                // pass 1: the row maximum over all 128 keys (both warpgroups of
-                // the tile compute it, identically), two 32-column chunks per
-                // TMEM wait and four running maxima
-                // (one 32-column chunk per TMEM wait here: this kernel's 18 warps
-                // leave 96 registers a thread)
+                // The row maximum over all 128 keys (both warpgroups of the tile
+                // compute it, identically) in two TMEM rounds of 64 columns: the
+                // other half's keys first, then this half's, which stay in
+                // registers for the probabilities.
                 float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                uint32_t v[2][32];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t va[32];
-                    tmem_ld_32x32b_x32(s_tm + 32 * c, va);
+                for (int round = 0; round < 2; ++round) {
+                    const int h = round == 0 ? 1 - hf : hf;
+                    tmem_ld_32x32b_x32(s_tm + 64 * h, v[0]);
+                    tmem_ld_32x32b_x32(s_tm + 64 * h + 32, v[1]);
                     tmem_ld_wait();
                     if (masked) {
 #pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            if (32 * c + e >= lim) va[e] = __float_as_uint(-INFINITY);
+                        for (int c = 0; c < 2; ++c)
+#pragma unroll
+                            for (int e = 0; e < 32; ++e)
+                                if (64 * h + 32 * c + e >= lim) v[c][e] = __float_as_uint(-INFINITY);
                     }
 #pragma unroll
-                    for (int e = 0; e < 32; e += 8) {
-                        m4[0] = fmax3(m4[0], __uint_as_float(va[e]), __uint_as_float(va[e + 1]));
-                        m4[1] = fmax3(m4[1], __uint_as_float(va[e + 2]), __uint_as_float(va[e + 3]));
-                        m4[2] = fmax3(m4[2], __uint_as_float(va[e + 4]), __uint_as_float(va[e + 5]));
-                        m4[3] = fmax3(m4[3], __uint_as_float(va[e + 6]), __uint_as_float(va[e + 7]));
-                    }
+                    for (int c = 0; c < 2; ++c)
+#pragma unroll
+                        for (int e = 0; e < 32; e += 8) {
+                            m4[0] = fmax3(m4[0], __uint_as_float(v[c][e]), __uint_as_float(v[c][e + 1]));
+                            m4[1] = fmax3(m4[1], __uint_as_float(v[c][e + 2]), __uint_as_float(v[c][e + 3]));
+                            m4[2] = fmax3(m4[2], __uint_as_float(v[c][e + 4]), __uint_as_float(v[c][e + 5]));
+                            m4[3] = fmax3(m4[3], __uint_as_float(v[c][e + 6]), __uint_as_float(v[c][e + 7]));
+                        }
                 }
+                // S_a is no longer read: the next block's Q K^T may overwrite it
+                // while these probabilities are computed
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(s_empty(a));
                 const float mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
                 const float mb = __fmul_rn(mx, p.sl2);
                 float alpha = 1.f;
@@ -471,6 +517,41 @@ __global__ void __launch_bounds__(AttnCore::kThreads, 1)
                     resc = true;
                 }
                 const float moff = m_run == -INFINITY ? 0.f : m_run;
+                // probabilities 2^(s log2(e)/sqrt(128) - m) of this half's 64
+                // keys and their sum, packed as bf16 pairs in place (pair e, e + 1
+                // into word e / 2, already read).  The exponent is one fused
+                // multiply-add: for the row's maximum it leaves only m's own
+                // rounding error, below 2^-12 while |m| < 4096.  Larger m
+                // (saturated inputs) take the product rounded first, as m was, so
+                // the maximum gives exactly 2^0.
+                const bool exact_max = fabsf(moff) >= 4096.f;
+                // eight partial sums, kept and added in pairs
+                float ls8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                const uint64_t sl2x2 = f32x2(p.sl2, p.sl2), negm2 = f32x2(-moff, -moff);
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t(&w)[32] = v[c];
+                    if (!exact_max) {
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) {
+                            float x0, x1;
+                            fma_f32x2(__uint_as_float(w[e]), __uint_as_float(w[e + 1]), sl2x2, negm2, x0, x1);
+                            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                            const int g = 2 * ((e >> 1) & 3);
+                            add_f32x2(ls8[g], ls8[g + 1], p0, p1);
+                            w[e >> 1] = pack_bf16x2(p0, p1);
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) {
+                            const float p0 = ex2_approx(__fmul_rn(__uint_as_float(w[e]), p.sl2) - moff);
+                            const float p1 = ex2_approx(__fmul_rn(__uint_as_float(w[e + 1]), p.sl2) - moff);
+                            const int g = 2 * ((e >> 1) & 3);
+                            add_f32x2(ls8[g], ls8[g + 1], p0, p1);
+                            w[e >> 1] = pack_bf16x2(p0, p1);
+                        }
+                    }
+                }
                 if (j > 0) {
                     // P_a and O_a are free once the previous block's P V is done
                     int w2 = 0;
@@ -481,72 +562,34 @@ __global__ void __launch_bounds__(AttnCore::kThreads, 1)
                         break;
                     }
                     tc_fence_after();
-                    if (__any_sync(0xffffffffu, resc)) {
-#pragma unroll 1
-                        for (int c = 0; c < 2; ++c) {
-                            uint32_t o[32];
-                            tmem_ld_32x32b_x32(o_tm + 32 * c, o);
-                            tmem_ld_wait();
-#pragma unroll
-                            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                            tmem_st_32x32b_x32(o_tm + 32 * c, o);
-                        }
-                        tmem_st_wait();
-                    }
                 }
-                // pass 2 (this half's 64 keys): probabilities 2^(s log2(e)/sqrt(128)
-                // - m), their sum, and P as bf16 in the 128-byte-swizzled K-major
-                // layout (box hf; 16-byte chunk k of row r at chunk k ^ (r % 8)).
-                // The exponent is one fused multiply-add: for the row's maximum it
-                // leaves only m's own rounding error, below 2^-12 while |m| <
-                // 4096.  Larger m (saturated inputs) take the product rounded
-                // first, as m was, so the maximum gives exactly 2^0.
-                const bool exact_max = fabsf(moff) >= 4096.f;
-                float ls4[4] = {0.f, 0.f, 0.f, 0.f};
-                uint32_t v[2][32];
-                tmem_ld_32x32b_x32(s_tm + 64 * hf, v[0]);
-                tmem_ld_32x32b_x32(s_tm + 64 * hf + 32, v[1]);
-                tmem_ld_wait();
-                // S_a is no longer read: the next block's Q K^T may overwrite it
-                // while these probabilities are computed
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(s_empty(a));
+                // P in the 128-byte-swizzled K-major layout (box hf; 16-byte chunk
+                // k of row r at chunk k ^ (r % 8))
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    const int col0 = 64 * hf + 32 * c;
-                    uint32_t(&w)[32] = v[c];
-                    uint32_t pk[16];
-                    if (masked) {
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            if (col0 + e >= lim) w[e] = __float_as_uint(-INFINITY);
-                    }
-                    if (!exact_max) {
-#pragma unroll
-                        for (int e = 0; e < 32; e += 2) {
-                            const float p0 = ex2_approx(fmaf(__uint_as_float(w[e]), p.sl2, -moff));
-                            const float p1 = ex2_approx(fmaf(__uint_as_float(w[e + 1]), p.sl2, -moff));
-                            ls4[(e >> 1) & 3] += p0 + p1;
-                            pk[e >> 1] = pack_bf16x2(p0, p1);
-                        }
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 32; e += 2) {
-                            const float p0 = ex2_approx(__fmul_rn(__uint_as_float(w[e]), p.sl2) - moff);
-                            const float p1 = ex2_approx(__fmul_rn(__uint_as_float(w[e + 1]), p.sl2) - moff);
-                            ls4[(e >> 1) & 3] += p0 + p1;
-                            pk[e >> 1] = pack_bf16x2(p0, p1);
-                        }
-                    }
+                for (int c = 0; c < 2; ++c)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint32_t chunk = static_cast<uint32_t>(c * 4 + kk);
-                        st_shared_v4(p_row + ((chunk ^ swz) << 4), pk[4 * kk], pk[4 * kk + 1],
-                                     pk[4 * kk + 2], pk[4 * kk + 3]);
+                        st_shared_v4(p_row + ((chunk ^ swz) << 4), v[c][4 * kk], v[c][4 * kk + 1],
+                                     v[c][4 * kk + 2], v[c][4 * kk + 3]);
                     }
+                // O_a is rescaled (rarely) with the scores' registers free
+                if (j > 0 && __any_sync(0xffffffffu, resc)) {
+#pragma unroll 1
+                    for (int c = 0; c < 2; ++c) {
+                        uint32_t o[32];
+                        tmem_ld_32x32b_x32(o_tm + 32 * c, o);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                        tmem_st_32x32b_x32(o_tm + 32 * c, o);
+                    }
+                    tmem_st_wait();
                 }
-                lsum = lsum * alpha + ((ls4[0] + ls4[1]) + (ls4[2] + ls4[3]));
+                add_f32x2(ls8[0], ls8[1], ls8[2], ls8[3]);
+                add_f32x2(ls8[4], ls8[5], ls8[6], ls8[7]);
+                add_f32x2(ls8[0], ls8[1], ls8[4], ls8[5]);
+                lsum = lsum * alpha + (ls8[0] + ls8[1]);
                 fence_proxy_async_smem();
                 tc_fence_before();
                 __syncwarp();
