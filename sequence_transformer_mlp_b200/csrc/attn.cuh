@@ -142,7 +142,7 @@ struct AttnCore {
     static constexpr int kStages = 3;
     static constexpr int kQOff = 0, kPOff = 2 * kTileBytes, kKVOff = 4 * kTileBytes;
     static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
-    static constexpr int kSmemBytes = kBarOff + 256 + 1024;
+    static constexpr int kSmemBytes = kBarOff + 512 + 1024;
     // Q K^T in fp16 (the block's projections store Q and K as fp16: three more
     // mantissa bits than bf16 where the scores' rounding matters most) or bf16
     static constexpr uint32_t kIdescSf16 = make_idesc_f16(128, 128, false, false);
@@ -220,7 +220,12 @@ __global__ void __launch_bounds__(AttnCore::kThreads, 1)
     auto p_full = [&](int a) { return bar0 + 16u + 8u * (2 * S + 4 + a); };
     auto pv_done = [&](int a) { return bar0 + 16u + 8u * (2 * S + 6 + a); };
     const uint32_t drain_bar = bar0 + 16u + 8u * (2 * S + 8);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 + 2 * S + 9);
+    // the two warps holding rows 32 q .. 32 q + 31 of tile a meet at the end of
+    // an item: their row sums are published (x_full), then read (x_read)
+    auto x_full = [&](int a, int q) { return bar0 + 16u + 8u * (2 * S + 9 + 4 * a + q); };
+    auto x_read = [&](int a, int q) { return bar0 + 16u + 8u * (2 * S + 17 + 4 * a + q); };
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 + 2 * S + 25);
+    static_assert(8 * (2 + 2 * S + 25) + 8 <= 512, "barrier area");
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -239,6 +244,11 @@ __global__ void __launch_bounds__(AttnCore::kThreads, 1)
             mbar_init(pv_done(a), 1);
         }
         mbar_init(drain_bar, 1);
+        for (int a = 0; a < 2; ++a)
+            for (int q = 0; q < 4; ++q) {
+                mbar_init(x_full(a, q), 2);
+                mbar_init(x_read(a, q), 2);
+            }
         *abort_flag = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
@@ -444,8 +454,7 @@ __global__ void __launch_bounds__(AttnCore::kThreads, 1)
         const uint32_t p_row = p_box + r * 128;
         const uint32_t p_row_other = ps + a * C::kTileBytes + (1 - hf) * 16384 + r * 128;
         const uint32_t swz = static_cast<uint32_t>(r & 7);
-        const uint32_t bar_id = 1u + static_cast<uint32_t>(a * 4 + q);  // the row's two warps
-        uint32_t s_cnt = 0, pv_cnt = 0;
+        uint32_t s_cnt = 0, pv_cnt = 0, xn = 0;  // xn: end-of-item meetings so far
         bool ok = true;
         for (int rd = 0; rd < rounds && ok; ++rd) {
             const int k = C::item_index(p, rd, cta, G);
@@ -606,11 +615,25 @@ __global__ void __launch_bounds__(AttnCore::kThreads, 1)
             // the last P V has read P: each half leaves its partial sum in its
             // own P row, the row's two warps meet, read the other's, and meet
             // again before either writes P of the next item there
+            // (bounded meetings on mbarriers, so that a partner which left on a
+            // timeout cannot hold the other warp)
+            auto meet = [&](uint32_t bar) {
+                __syncwarp();
+                int wm = 0;
+                if (lane == 0) {
+                    mbar_arrive(bar);
+                    wm = mbar_wait(bar, xn & 1u, abort_flag) ? 1 : 0;
+                }
+                wm = __shfl_sync(0xffffffffu, wm, 0);
+                __syncwarp();
+                return wm != 0;
+            };
             asm volatile("st.shared.f32 [%0], %1;" ::"r"(p_row), "f"(lsum) : "memory");
-            asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
+            if (!meet(x_full(a, q))) break;
             float lo;
             asm volatile("ld.shared.f32 %0, [%1];" : "=f"(lo) : "r"(p_row_other) : "memory");
-            asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
+            if (!meet(x_read(a, q))) break;
+            ++xn;
             const float inv = 1.f / (hf == 0 ? lsum + lo : lo + lsum);
             const bool row_ok = qrow <= it.qlast;
             __nv_bfloat16* orow = p.O + static_cast<long long>(qrow) * p.ldo + it.h * 128 + 64 * hf;
