@@ -19,7 +19,7 @@ import torch
 
 import sequence_transformer_mlp_b200 as T
 from oracle import attention as OA
-from workloads import AttnWorkload, TSP_ATTN, cover_rows, make_attn_inputs, make_qkv
+from workloads import ATTN_WORKLOADS, AttnWorkload, cover_rows, make_attn_inputs, make_qkv
 
 pytestmark = pytest.mark.gpu
 
@@ -143,14 +143,15 @@ def test_block_small_shapes(n, d, heads, P, causal, w_std):
     check(np64(Y), ref, f"block n={n} d={d} P={P} causal={causal}")
 
 
-def test_block_long_context_sampled_rows():
-    """The TSP attention workload (32768 tokens in 8 sequence shards of 4096,
-    32 heads of 128 in 8 parameter shards, causal), in the launch configuration
-    the benchmark times.  Rows: one seeded row in each of the 128 blocks of 256
-    tokens (every query-tile pair of every sequence shard, so every work item's
-    ring start and diagonal position), plus each sequence shard's first and
-    last row."""
-    wl = TSP_ATTN
+@pytest.mark.parametrize("name", sorted(ATTN_WORKLOADS))
+def test_block_long_context_sampled_rows(name):
+    """The TSP attention workloads (32768 tokens in 8 sequence shards of 4096,
+    32 heads of 128 in 8 parameter shards; causal, and the same without the
+    mask), in the launch configuration the benchmark times.  Rows: one seeded
+    row in each of the 128 blocks of 256 tokens (every query-tile pair of every
+    sequence shard, so every work item's ring start and, with the mask, its
+    diagonal position), plus each sequence shard's first and last row."""
+    wl = ATTN_WORKLOADS[name]
     inp = make_attn_inputs(wl)
     dev = {k: v.cuda() for k, v in inp.items()}
     Y = T.attn_forward(dev["X"], dev["Wq"], dev["Wk"], dev["Wv"], dev["Wo"], wl.heads, wl.P,
