@@ -29,7 +29,9 @@
  * (torch.nn.Linear stores the transpose of each weight.)
  * TSP_DT_BF16: X, weights, dY, Y and dX are bfloat16; every product
  *   accumulates in fp32; the hidden activation is rounded to bf16 once before
- *   the down projection; weight gradients are fp32.
+ *   the down projection; in the backward, the activation's derivative factors
+ *   and dG (dU) are rounded to bf16 before their products; weight gradients
+ *   are fp32.
  * TSP_DT_F32: everything fp32 (no TF32), plain or gated.
  *
  * Ownership.  The caller owns every buffer.  Pointers are device pointers on
@@ -250,15 +252,15 @@ TSP_API tsp_status_t tsp_mlp_workspace_size(int64_t n_tokens, int64_t d_model, i
  * the Math": the plain block).  tsp_mlp_forward_train writes, besides Y, the
  * activations and the activation's derivative factors at every hidden unit:
  *   H  = h(X)                    bf16 [n_tokens][d_ff]  (as the forward's)
- *   S1 = SiLU(G)  (SwiGLU)  or  GeLU'(Z) (GeLU)          fp32 [n_tokens][d_ff]
- *   S2 = U SiLU'(G)  (SwiGLU only)                       fp32 [n_tokens][d_ff]
- * with G = X.W_gate, U = X.W_up, Z = X.A, SiLU'(g) = s (1 + g (1 - s)),
- * s = sigmoid(g), GeLU'(z) = Phi(z) + z phi(z); and tsp_mlp_backward_saved
- * forms dU = dH S1 and dG = dH S2 (GeLU: dG = dH S1) in the epilogue of the
- * dH product, so dH is never stored.  The factors are evaluated exactly as
- * tsp_mlp_backward_ex evaluates them from its recomputed G and U, so dX,
- * dW_gate and dW_up are bit-identical to its results; dW_down uses the
- * forward's H.
+ *   S1 = SiLU(G)  (SwiGLU)  or  GeLU'(Z) (GeLU)          bf16 [n_tokens][d_ff]
+ *   S2 = U SiLU'(G)  (SwiGLU only)                       bf16 [n_tokens][d_ff]
+ * with G = X.W_gate, U = X.W_up, Z = X.A (fp32 accumulations), SiLU'(g) =
+ * s (1 + g (1 - s)), s = sigmoid(g), GeLU'(z) = Phi(z) + z phi(z), each factor
+ * evaluated in fp32 and rounded to bf16; and tsp_mlp_backward_saved forms
+ * dU = dH S1 and dG = dH S2 (GeLU: dG = dH S1) in the epilogue of the dH
+ * product, so dH is never stored.  tsp_mlp_backward_ex evaluates and rounds
+ * the factors the same way from its recomputed G and U, so dX, dW_gate and
+ * dW_up are bit-identical to its results; dW_down uses the forward's H.
  *
  * The saved buffer is opaque to the caller: H (row-major), then S1, then S2
  * (each over whole 32-row blocks, in the layout the two epilogues access

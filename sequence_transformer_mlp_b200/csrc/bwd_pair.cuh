@@ -28,6 +28,10 @@ __device__ __forceinline__ float gelu_grad_rn(float z, float cdf) {
     const float pdf = __fmul_rn(0.39894228040143267794f, __expf(__fmul_rn(__fmul_rn(-0.5f, z), z)));
     return __fmaf_rn(z, pdf, cdf);
 }
+// A factor as both backward paths use it: rounded to bf16 (nearest even, the
+// rounding of pack_bf16x2, which stores the training forward's factors) and
+// widened back to float.
+__device__ __forceinline__ float bf16_round(float x) { return __uint_as_float(pack_bf16x2(x, 0.0f) << 16); }
 
 // ============================================================================
 // Paired weight gradients (see Wgrad): both operands MN-major, K = tokens.
@@ -109,8 +113,10 @@ struct WgradPair {
 //   SwiGLU: H = SiLU(G) U,  dU = dH SiLU(G),  dG = dH U SiLU'(G)   (bf16)
 //   GeLU:   H = GeLU(G),    dG = dH GeLU'(G)                        (bf16)
 // with SiLU'(g) = s (1 + g (1 - s)), s = sigmoid(g), and GeLU'(z) = Phi(z) +
-// z phi(z): the derivatives of the forward definition (helpers above).  dH stays fp32, so
-// the only roundings are those of H, dG and dU to bf16.
+// z phi(z): the derivatives of the forward definition (helpers above).  dH stays
+// fp32; the factors SiLU(G), U SiLU'(G) and GeLU'(G) are rounded to bf16 before
+// the products, as the training forward saves them (train_pair.cuh), and H,
+// dG and dU are rounded to bf16.
 struct DhParams {
     CUtensorMap tmDY;  // dY [n][d], box {64, 128}
     CUtensorMap tmD;   // W_down / B [f][d], box {64, 128} (K-major: rows are hidden units)
@@ -297,8 +303,9 @@ struct BwdGateUpPair {
                         const float sg = sigmoid_rn(gv);
                         const float si = __fmul_rn(gv, sg);
                         h[j] = si * uv;
-                        duv[j] = dh[2 * i + j] * si;
-                        dgv[j] = dh[2 * i + j] * swiglu_gate_factor(gv, uv, sg);
+                        // the factors rounded to bf16, as the training forward saves them
+                        duv[j] = dh[2 * i + j] * bf16_round(si);
+                        dgv[j] = dh[2 * i + j] * bf16_round(swiglu_gate_factor(gv, uv, sg));
                     }
                     ph[i] = pack_bf16x2(h[0], h[1]);
                     pg[i] = pack_bf16x2(dgv[0], dgv[1]);
@@ -316,7 +323,7 @@ struct BwdGateUpPair {
                         const float z = __uint_as_float(g[2 * i + j]);
                         const float cdf = gelu_cdf_rn(z);
                         h[j] = z * cdf;
-                        dgv[j] = dh[2 * i + j] * gelu_grad_rn(z, cdf);
+                        dgv[j] = dh[2 * i + j] * bf16_round(gelu_grad_rn(z, cdf));
                     }
                     ph[i] = pack_bf16x2(h[0], h[1]);
                     pg[i] = pack_bf16x2(dgv[0], dgv[1]);

@@ -4,20 +4,22 @@
 // The recompute backward (bwd_pair.cuh) runs the gate/up projection a second
 // time to get G and U back.  Here the forward's gate/up epilogue, which has G
 // and U in tensor memory anyway, also writes the activation's derivative
-// factors in fp32, and the dH GEMM's epilogue turns dH into dG (and dU) with
-// them directly:
+// factors, rounded to bf16 like the other saved activation H, and the dH
+// GEMM's epilogue turns dH into dG (and dU) with them directly:
 //   SwiGLU: S1 = SiLU(G),  S2 = U SiLU'(G)   dU = dH S1,  dG = dH S2
 //   GeLU:   S1 = GeLU'(Z)                     dG = dH S1
 // with SiLU'(g) = s (1 + g (1 - s)), s = sigmoid(g), GeLU'(z) = Phi(z) +
-// z phi(z) -- the derivatives of the forward definition, evaluated by the
-// recompute backward's own helpers (bwd_pair.cuh, every rounding explicit),
-// so dG and dU come out bit for bit the same.  dH itself is never stored.
+// z phi(z) -- the derivatives of the forward definition, evaluated in fp32
+// by the recompute backward's own helpers (bwd_pair.cuh, every rounding
+// explicit) and rounded to bf16 there too, so dG and dU come out bit for bit
+// the same.  dH itself is never stored.
 //
 // The factors are private to this pair, so their layout follows the
 // epilogues' access, where a thread owns a row and a warp 32 consecutive rows:
-// factor (r, c) sits at ((r / 32) * ld + c) * 32 + r % 32, each 32-row block
-// column-interleaved.  A warp then reads or writes one column of its 32 rows
-// as 128 contiguous bytes, instead of 32 rows' 16-byte pieces.
+// the pair of factors (r, c), (r, c + 1) (c even) is one bf16x2 word, at word
+// ((r / 32) * ld / 2 + c / 2) * 32 + r % 32 -- each 32-row block interleaved
+// by column pairs.  A warp then reads or writes two columns of its 32 rows as
+// 128 contiguous bytes, instead of 32 rows' 4-byte pieces.
 #pragma once
 
 #include "bwd_pair.cuh"
@@ -28,13 +30,14 @@ namespace tspmlp {
 // Gate/up projection (as FwdHiddenPair) whose epilogue also keeps S1 (S2).
 template <int ACT>
 struct FwdHiddenSaveParams : FwdHidden<ACT>::Params {
-    float* S1;  // fp32, 32-row blocks of ldh columns, column-interleaved
-    float* S2;  // (SwiGLU)
+    uint32_t* S1;  // bf16x2 words, 32-row blocks of ldh columns, interleaved by column pairs
+    uint32_t* S2;  // (SwiGLU)
 };
 
-// Offset of factor (r, c) in the 32-row-block layout with ld columns.
-__device__ __forceinline__ long long factor_index(int r, int c, long long ld) {
-    return (static_cast<long long>(r >> 5) * ld + c) * 32 + (r & 31);
+// Word of the factor pair (r, c), (r, c + 1), c even, in the 32-row-block
+// layout with ld (even) columns.
+__device__ __forceinline__ long long factor_word(int r, int c, long long ld) {
+    return (static_cast<long long>(r >> 5) * (ld >> 1) + (c >> 1)) * 32 + (r & 31);
 }
 
 template <int ACT>
@@ -44,11 +47,13 @@ struct FwdHiddenSavePair : FwdHiddenPair<ACT> {
     using Tile = typename Base::Tile;
     static constexpr const char* kName = ACT == 1 ? "fwd_hidden_swiglu_save" : "fwd_hidden_gelu_save";
 
-    // the thread's 32 consecutive factors of one row: a column 32 floats apart
-    __device__ static void store_factors(float* dst, const uint32_t (&v)[32], int valid) {
+    // the thread's 32 consecutive factors of one row (fp32 bits), rounded to
+    // bf16 in pairs: a column pair 32 words apart
+    __device__ static void store_factors(uint32_t* dst, const uint32_t (&v)[32], int valid) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-            if (i < valid) dst[32 * i] = __uint_as_float(v[i]);
+        for (int i = 0; i < 16; ++i)
+            if (2 * i < valid)
+                dst[32 * i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
     }
 
     __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t rank, uint32_t acc,
@@ -85,8 +90,8 @@ struct FwdHiddenSavePair : FwdHiddenPair<ACT> {
                     pk[i] = pack_bf16x2(__uint_as_float(g[2 * i]), __uint_as_float(g[2 * i + 1]));
                 warp_store_16x32(stg, p.H + off0 + c0, p.ldh, nrows, pk, valid, lane);
                 if (row_ok) {
-                    store_factors(p.S1 + factor_index(r, c0, p.ldh), s1, valid);
-                    store_factors(p.S2 + factor_index(r, c0, p.ldh), s2, valid);
+                    store_factors(p.S1 + factor_word(r, c0, p.ldh), s1, valid);
+                    store_factors(p.S2 + factor_word(r, c0, p.ldh), s2, valid);
                 }
             } else {
                 tmem_ld_wait();
@@ -102,7 +107,7 @@ struct FwdHiddenSavePair : FwdHiddenPair<ACT> {
                 for (int i = 0; i < 16; ++i)
                     pk[i] = pack_bf16x2(__uint_as_float(g[2 * i]), __uint_as_float(g[2 * i + 1]));
                 warp_store_16x32(stg, p.H + off0 + c0, p.ldh, nrows, pk, valid, lane);
-                if (row_ok) store_factors(p.S1 + factor_index(r, c0, p.ldh), s1, valid);
+                if (row_ok) store_factors(p.S1 + factor_word(r, c0, p.ldh), s1, valid);
             }
         }
     }
@@ -112,9 +117,9 @@ struct FwdHiddenSavePair : FwdHiddenPair<ACT> {
 // dH = dY . W_down[c..]^T (as DhPair), whose epilogue applies the saved
 // factors and writes dG (dU) in bf16 instead of storing dH.
 struct DhFactorParams : DhParams {
-    const float* S1;  // saved factors (32-row-block layout) from the chunk's first column
-    const float* S2;  // (SwiGLU)
-    long long lds;    // columns of the saved layout (d_ff)
+    const uint32_t* S1;  // saved factors (bf16x2 words, 32-row-block layout) from the chunk's first column
+    const uint32_t* S2;  // (SwiGLU)
+    long long lds;       // columns of the saved layout (d_ff, even)
     __nv_bfloat16* dG;  // [n][width] at pitch ld
     __nv_bfloat16* dU;  // [n][width] (SwiGLU)
 };
@@ -126,11 +131,15 @@ struct DhFactorPair : DhPair<ACT> {
     using Tile = typename Base::Tile;
     static constexpr const char* kName = ACT == 1 ? "bwd_dh_factor_swiglu" : "bwd_dh_factor_gelu";
 
-    // the thread's 32 consecutive factors of one row (a column 32 floats
-    // apart), zero beyond valid
-    __device__ static void load_factors(const float* src, int valid, float (&v)[32]) {
+    // the thread's 32 consecutive factors of one row (a column pair 32 words
+    // apart), widened to float; zero from the first pair beyond valid
+    __device__ static void load_factors(const uint32_t* src, int valid, float (&v)[32]) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = i < valid ? src[32 * i] : 0.0f;
+        for (int i = 0; i < 16; ++i) {
+            const uint32_t w = 2 * i < valid ? src[32 * i] : 0u;
+            v[2 * i] = __uint_as_float(w << 16);
+            v[2 * i + 1] = __uint_as_float(w & 0xffff0000u);
+        }
     }
 
     __device__ static void epilogue(const Params& p, const Tile& ti, uint32_t rank, uint32_t acc,
@@ -148,7 +157,7 @@ struct DhFactorPair : DhPair<ACT> {
             const bool live = row_ok && valid > 0;
             float s1[32], s2[32];
             if (live) {
-                const long long so = factor_index(row, c0, p.lds);
+                const long long so = factor_word(row, c0, p.lds);
                 load_factors(p.S1 + so, valid, s1);
                 if (ACT == 1) load_factors(p.S2 + so, valid, s2);
             } else {

@@ -637,8 +637,8 @@ template <int ACT>
 tsp_status_t fwd_pass_bf16(const void* X, const void* Wg, const void* Wu, const void* Wd,
                            int64_t n, int64_t d, int64_t f, const SegGeom& g, int64_t width,
                            int mode, __nv_bfloat16* H, float* acc, void* Y, cudaStream_t st,
-                           int dev, int sms, int rot_P = 0, float* S1 = nullptr,
-                           float* S2 = nullptr, char* split_area = nullptr) {
+                           int dev, int sms, int rot_P = 0, uint32_t* S1 = nullptr,
+                           uint32_t* S2 = nullptr, char* split_area = nullptr) {
     using K1 = FwdHidden<ACT>;
     using K2 = DownAccum<true, 1>;
     typename K1::Params p1;
@@ -913,9 +913,9 @@ tsp_status_t forward_bf16(const void* X, const void* Wg, const void* Wu, const v
 // keeps those factors (train_pair.cuh) so that the backward need not run the
 // gate/up projection again.
 
-// Saved activations: H (bf16 [n][f]), then the fp32 factor regions S1 (and
+// Saved activations: H (bf16 [n][f]), then the bf16 factor regions S1 (and
 // S2 for SwiGLU), each of whole 32-row blocks of f columns (the layout of
-// train_pair.cuh), every region 256-byte aligned.
+// train_pair.cuh: bf16x2 words of column pairs), every region 256-byte aligned.
 struct SavedLayout {
     size_t h = 0, s = 0;
     int nfac = 1;
@@ -930,7 +930,7 @@ struct SavedLayout {
 SavedLayout saved_layout(int64_t n, int64_t f, tsp_act_t act) {
     SavedLayout l;
     l.h = align256(static_cast<size_t>(n) * f * 2);
-    l.s = align256(static_cast<size_t>((n + 31) / 32 * 32) * f * 4);
+    l.s = align256(static_cast<size_t>((n + 31) / 32 * 32) * f * 2);
     l.nfac = act == TSP_ACT_SWIGLU ? 2 : 1;
     return l;
 }
@@ -953,8 +953,8 @@ tsp_status_t forward_train_bf16(const void* X, const void* Wg, const void* Wu, c
     const SavedLayout sl = saved_layout(n, f, ACT == 1 ? TSP_ACT_SWIGLU : TSP_ACT_GELU);
     char* base = static_cast<char*>(saved);
     auto* H = reinterpret_cast<__nv_bfloat16*>(base);
-    auto* S1 = reinterpret_cast<float*>(base + sl.h);
-    float* S2 = ACT == 1 ? reinterpret_cast<float*>(base + sl.h + sl.s) : nullptr;
+    auto* S1 = reinterpret_cast<uint32_t*>(base + sl.h);
+    uint32_t* S2 = ACT == 1 ? reinterpret_cast<uint32_t*>(base + sl.h + sl.s) : nullptr;
     const int64_t fs = f / P, rg = train_row_group(n, f);
     const size_t xe = static_cast<size_t>(d) * 2;
     for (int64_t r0 = 0; r0 < n; r0 += rg) {
@@ -963,10 +963,10 @@ tsp_status_t forward_train_bf16(const void* X, const void* Wg, const void* Wu, c
         void* Yg = static_cast<char*>(Y) + r0 * xe;
         const SegGeom g = seg_all_rows(rows, P, fs, 0);
         // row groups start on 256-row boundaries, so a group's factors begin
-        // at the same offset r0 x f as its rows of H
-        const int64_t ho = r0 * f;
+        // at element r0 x f, as its rows of H: word r0 x f / 2
+        const int64_t ho = r0 * f, so = ho / 2;
         TSP_TRY(fwd_pass_bf16<ACT>(Xg, Wg, Wu, Wd, rows, d, f, g, f, /*mode direct*/ 3, H + ho,
-                                   nullptr, Yg, st, dev, sms, 0, S1 + ho, S2 ? S2 + ho : nullptr,
+                                   nullptr, Yg, st, dev, sms, 0, S1 + so, S2 ? S2 + so : nullptr,
                                    base + sl.split_offset()));
     }
     return TSP_OK;
@@ -1090,8 +1090,8 @@ BwdPlan plan_backward_for(int64_t n, int64_t d, int64_t f, int P, tsp_act_t act,
 // Activations kept by the training forward (see SavedLayout), row pitch ld.
 struct SavedAct {
     const __nv_bfloat16* H;
-    const float* S1;
-    const float* S2;
+    const uint32_t* S1;  // bf16x2 words (train_pair.cuh)
+    const uint32_t* S2;
     int64_t ld;
 };
 
@@ -1126,8 +1126,8 @@ tsp_status_t backward_bf16(const void* X, const void* Wg, const void* Wu, const 
             p.col_base = static_cast<int>(cb);
             p.width = static_cast<int>(C);
             p.ld = C;
-            p.S1 = sv->S1 + cb * 32;  // column cb of every 32-row block
-            p.S2 = ACT == 1 ? sv->S2 + cb * 32 : nullptr;
+            p.S1 = sv->S1 + cb / 2 * 32;  // column cb (even) of every 32-row block
+            p.S2 = ACT == 1 ? sv->S2 + cb / 2 * 32 : nullptr;
             p.lds = sv->ld;
             p.dG = dGc;
             p.dU = dUc;
@@ -1588,8 +1588,8 @@ tsp_status_t tsp_mlp_backward_saved(const void* X, const void* Wg, const void* W
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const char* base = static_cast<const char*>(saved);
     const SavedAct sv{reinterpret_cast<const __nv_bfloat16*>(base),
-                      reinterpret_cast<const float*>(base + sl.h),
-                      act == TSP_ACT_SWIGLU ? reinterpret_cast<const float*>(base + sl.h + sl.s)
+                      reinterpret_cast<const uint32_t*>(base + sl.h),
+                      act == TSP_ACT_SWIGLU ? reinterpret_cast<const uint32_t*>(base + sl.h + sl.s)
                                             : nullptr,
                       f};
     if (act == TSP_ACT_SWIGLU)

@@ -166,15 +166,15 @@ def test_bad_pointers_are_rejected_before_any_device_call(lib):
 
 
 def test_training_pair_sizes(lib):
-    # saved activations: bf16 H, then fp32 S1 (and S2 for SwiGLU) over whole
+    # saved activations: bf16 H, then bf16 S1 (and S2 for SwiGLU) over whole
     # 32-row blocks, each region 256-byte aligned
     n, d, f, P = 4096, 4096, 14336, 8
     # (and the down projection's tail-split scratch, as the forward's workspace)
-    assert T.tsp_mlp_saved_size(n, d, f, P, "swiglu") == n * f * 2 + 2 * n * f * 4 + SPLIT
-    assert T.tsp_mlp_saved_size(n, d, f, P, "gelu") == n * f * 2 + n * f * 4 + SPLIT
+    assert T.tsp_mlp_saved_size(n, d, f, P, "swiglu") == n * f * 2 + 2 * n * f * 2 + SPLIT
+    assert T.tsp_mlp_saved_size(n, d, f, P, "gelu") == n * f * 2 + n * f * 2 + SPLIT
     # (the factor regions hold whole 32-row blocks)
     assert T.tsp_mlp_saved_size(3, 16, 8 * 3, 3, "swiglu") == \
-        _a256(3 * 24 * 2) + 2 * _a256(32 * 24 * 4) + SPLIT
+        _a256(3 * 24 * 2) + 2 * _a256(32 * 24 * 2) + SPLIT
     # the backward from saved activations needs only dG (dU) chunk buffers:
     # one chunk of all hidden units within the 1 GiB budget
     assert T.tsp_mlp_backward_saved_workspace_size(n, d, f, P, "swiglu") == 2 * n * f * 2
