@@ -111,7 +111,7 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
     PERIOD_S = 0.004
-    # clock-event reason bits (NVML): the ones a run is judged by
+    # clock-event reason bits (NVML): power capping, and the slowdowns that void a timing
     REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
                    "hw_thermal_slowdown": 0x40}
 
