@@ -6,7 +6,7 @@
   activations.
 - dX, dW_gate and dW_up are bit-identical to tsp_mlp_backward_ex's: the saved
   factors are the recompute backward's own expressions of the same fp32 G and
-  U, and dH is the same product.
+  U, rounded to bf16 the same way, and dH is the same product.
 - Every output meets the bf16 bar against the fp64 oracle (dW_down uses the
   forward's H, so it is compared with the oracle, not bit for bit).
 """
