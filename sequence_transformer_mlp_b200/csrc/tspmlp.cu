@@ -1186,9 +1186,11 @@ tsp_status_t backward_bf16(const void* X, const void* Wg, const void* Wu, const 
             p.out_col0 = 0;
             TSP_TRY((launch_pair<WgradPair<256, false>>(p, st, dev, sms)));
         }
-        if (sv && ACT == 1) {
+        if (ACT == 1) {
             // K4b + K5 in one launch (grad_pair.cuh): the input gradient's long
-            // tiles first, the weight gradients' short ones filling each pair
+            // tiles first, the weight gradients' short ones filling each pair.
+            // Both backward paths take it, so their dX, dW_gate and dW_up come
+            // from the same kernel.
             DgradWgradParams p;
             std::memset(&p, 0, sizeof(p));
             if (!tmap_bf16(&p.w.tmA, X, d, n, d, 64, 128, SW128) ||
@@ -1219,25 +1221,8 @@ tsp_status_t backward_bf16(const void* X, const void* Wg, const void* Wu, const 
             TSP_TRY(launch_pair<DgradWgradPair>(p, st, dev, sms));
             continue;
         }
-        // K4b: dW_gate (dW_up)[:, cb .. cb+C) = X^T . dG (dU)
-        if (ACT == 1) {
-            using K = Wgrad<256, true>;
-            typename K::Params p;
-            std::memset(&p, 0, sizeof(p));
-            if (!tmap_bf16(&p.tmA, X, d, n, d, 64, 64, SW128) ||
-                !tmap_bf16(&p.tmB0, dGc, C, n, C, 64, 64, SW128) ||
-                !tmap_bf16(&p.tmB1, dUc, C, n, C, 64, 64, SW128))
-                return TSP_ERR_CUDA;
-            p.ntok = static_cast<int>(n);
-            p.m_valid = static_cast<int>(d);
-            p.n_valid = static_cast<int>(C);
-            p.out0 = dWg;
-            p.out1 = dWu;
-            p.ldo = f;
-            p.out_row0 = 0;
-            p.out_col0 = static_cast<int>(cb);
-            TSP_TRY((launch_pair<WgradPair<256, true>>(p, st, dev, sms)));
-        } else {
+        // GeLU: K4b, dA[:, cb .. cb+C) = X^T . dG
+        {
             using K = Wgrad<128, false>;
             typename K::Params p;
             std::memset(&p, 0, sizeof(p));
@@ -1253,19 +1238,14 @@ tsp_status_t backward_bf16(const void* X, const void* Wg, const void* Wu, const 
             p.out_col0 = static_cast<int>(cb);
             TSP_TRY((launch_pair<WgradPair<128, false>>(p, st, dev, sms)));
         }
-        // K5: dX (+)= dG . W_gate[:, chunk]^T (+ dU . W_up[:, chunk]^T)
+        // GeLU: K5, dX (+)= dG . A[:, chunk]^T
         {
-            constexpr int NS = ACT == 1 ? 2 : 1;
-            using K = DownAccum<false, NS>;
+            using K = DownAccum<false, 1>;
             typename K::Params p;
             std::memset(&p, 0, sizeof(p));
             p.g = seg_all_rows(n, P, fs, cb);
-            p.n_out = static_cast<int>(d);
             if (!tmap_bf16(&p.tmA0, dGc, C, n, C, 64, 128, SW128) ||
                 !tmap_bf16(&p.tmB0, Wg, f, d, f, 64, 128, SW128))
-                return TSP_ERR_CUDA;
-            if (ACT == 1 && (!tmap_bf16(&p.tmA1, dUc, C, n, C, 64, 128, SW128) ||
-                             !tmap_bf16(&p.tmB1, Wu, f, d, f, 64, 128, SW128)))
                 return TSP_ERR_CUDA;
             p.kdim = static_cast<int>(C);
             p.n_out = static_cast<int>(d);
@@ -1274,7 +1254,7 @@ tsp_status_t backward_bf16(const void* X, const void* Wg, const void* Wu, const 
             p.ldacc = d;
             p.out = static_cast<__nv_bfloat16*>(dX);
             p.ldo = d;
-            TSP_TRY((launch_pair<DownAccumPair<false, NS, 256>>(p, st, dev, sms)));
+            TSP_TRY((launch_pair<DownAccumPair<false, 1, 256>>(p, st, dev, sms)));
         }
     }
     return TSP_OK;
