@@ -35,6 +35,24 @@ def test_header_declares_the_api():
             "tsp_mlp_backward_saved_workspace_size"} <= syms
 
 
+def test_header_is_plain_c(tmp_path):
+    """The boundary is a C ABI: the header compiles as strict C99 on its own
+    (no C++ or CUDA types in the declarations) and as C++."""
+    import shutil
+    import subprocess
+    src = tmp_path / "use_header.c"
+    src.write_text('#include "tspmlp.h"\nint main(void) { return (int)TSP_OK; }\n')
+    inc = os.path.join(ROOT, "include")
+    for cc, std in (("gcc", "-std=c99"), ("g++", "-std=c++17")):
+        if shutil.which(cc) is None:
+            pytest.skip(f"{cc} not found")
+        flags = [std, "-Wall", "-Wextra", "-Werror", "-pedantic"]
+        if cc == "g++":
+            flags += ["-x", "c++"]
+        subprocess.run([cc, *flags, "-I", inc, "-c", str(src), "-o", str(tmp_path / "use.o")],
+                       check=True)
+
+
 def test_library_exports_every_declared_symbol(lib):
     for name in declared_symbols():
         assert hasattr(lib, name), name
